@@ -1,0 +1,172 @@
+// Prompt-block pruning: representative keys and relevance top-C.
+//
+// Focus-dLLM summary page, "方法步骤详情" (method steps), step (4): the prompt is cut
+// into contiguous blocks, each represented by the mean of its keys; a relevance score
+// R_b of the active queries to each block keeps the top-C blocks. Reading fixed by the
+// build's specification: R_b^h = mean over the active queries and the query heads of
+// KV group h of q . kbar_b / sqrt(d), which equals qbar_h . kbar_b / sqrt(d).
+#include "focus_common.cuh"
+#include "topk.cuh"
+
+namespace focus {
+
+// kbar[bh, j, :] = mean of K[bh, j*bs : min(P, (j+1)*bs), :]. One CTA per (block, head);
+// 16-byte coalesced loads (one row = CH threads), fp32 accumulation, shared-memory reduction.
+template <int D>
+__global__ void __launch_bounds__(256) block_means_kernel(const __nv_bfloat16* __restrict__ K, int L, int P, int bs,
+                                                          int nb, float* __restrict__ kbar) {
+  constexpr int CH = D / 8;
+  constexpr int RL = 256 / CH;            // rows in flight per pass
+  __shared__ float red[RL][D + 4];
+  const int blk = blockIdx.x, bh = blockIdx.y;
+  const int c = threadIdx.x % CH, rl = threadIdx.x / CH;
+  const int r0 = blk * bs;
+  const int size = min(bs, P - r0);
+  const uint4* src = reinterpret_cast<const uint4*>(K + (static_cast<size_t>(bh) * L + r0) * D) + c;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int r = rl; r < size; r += RL) {
+    const uint4 v = __ldg(src + static_cast<size_t>(r) * CH);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      acc[2 * e] += f.x;
+      acc[2 * e + 1] += f.y;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[rl][c * 8 + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float s = 0.f;
+#pragma unroll 8
+    for (int q = 0; q < RL; ++q) s += red[q][threadIdx.x];
+    kbar[(static_cast<size_t>(bh) * nb + blk) * D + threadIdx.x] = s / static_cast<float>(size);
+  }
+}
+
+constexpr int kSelectThreads = 512;
+
+// One CTA per (sequence, KV head): qbar, R over all blocks, top-C.
+template <int D>
+__global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
+    const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ n_active, const float* __restrict__ kbar, int Hq,
+    int Hkv, int acap, int nb, int C, int32_t* __restrict__ blocks, float* __restrict__ scores) {
+  constexpr int PARTS = kSelectThreads / D;
+  extern __shared__ float s_R[];           // [nb]
+  __shared__ float s_part[PARTS][D];
+  __shared__ float s_qbar[D];
+  __shared__ TopkShared tk;
+  const int bh = blockIdx.x;
+  const int b = bh / Hkv, h = bh % Hkv;
+  const int g = Hq / Hkv;
+  const int A = n_active[b];
+  const int dim = threadIdx.x % D, part = threadIdx.x / D;
+  float acc = 0.f;
+  const int rows = g * A;
+  for (int r = part; r < rows; r += PARTS) {
+    const int hq = h * g + r / A, i = r % A;
+    acc += __bfloat162float(Q[((static_cast<size_t>(b) * Hq + hq) * acap + i) * D + dim]);
+  }
+  s_part[part][dim] = acc;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float s = 0.f;
+#pragma unroll
+    for (int p = 0; p < PARTS; ++p) s += s_part[p][threadIdx.x];
+    s_qbar[threadIdx.x] = rows > 0 ? s / static_cast<float>(rows) : 0.f;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int LANES = D / 4;             // float4 per lane
+  const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+  float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane < LANES) qv = reinterpret_cast<const float4*>(s_qbar)[lane];
+  const float* kb = kbar + static_cast<size_t>(bh) * nb * D;
+  for (int j = warp; j < nb; j += kSelectThreads / 32) {
+    float p = 0.f;
+    if (lane < LANES) {
+      const float4 kv = __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D) + lane);
+      p = qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+    if (lane == 0) {
+      const float R = p * inv_sqrt_d;
+      s_R[j] = R;
+      if (scores) scores[static_cast<size_t>(bh) * nb + j] = R;
+    }
+  }
+  __syncthreads();
+  block_topk_ascending([&](int i) { return float_order_key(s_R[i]); }, nb, C, blocks + static_cast<size_t>(bh) * C, C,
+                       tk);
+}
+
+}  // namespace focus
+
+using namespace focus;
+
+extern "C" int focus_block_means(const focus_bf16* K, int B, int Hkv, int L, int d, int P, int bs, float* kbar,
+                                 void* stream) {
+  FOCUS_CHECK_ARG(K && kbar, "null pointer argument");
+  FOCUS_CHECK_ARG(B >= 0 && Hkv >= 1 && L >= 1 && 1 <= P && P <= L && bs >= 1, "bad sizes (P=%d L=%d bs=%d)", P, L, bs);
+  FOCUS_CHECK_ARG(aligned16(K) && aligned16(kbar), "tensors must be 16-byte aligned");
+  if (d != 64 && d != 128) {
+    set_error("head dim %d unsupported (64 or 128)", d);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
+  if (B == 0) return FOCUS_OK;
+  const int nb = (P + bs - 1) / bs;
+  FOCUS_CHECK_ARG(static_cast<long long>(B) * Hkv < 65536, "B*Hkv must be < 65536");
+  dim3 grid(nb, B * Hkv);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    block_means_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(K), L, P, bs, nb, kbar);
+  else
+    block_means_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(K), L, P, bs, nb, kbar);
+  note_launch();
+  return launch_status("block_means kernel");
+}
+
+extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_active, const float* kbar, int B,
+                                  int Hq, int Hkv, int d, int acap, int nb, int C, int32_t* blocks, float* scores_opt,
+                                  void* stream) {
+  FOCUS_CHECK_ARG(Q_active && n_active && kbar && blocks, "null pointer argument");
+  FOCUS_CHECK_ARG(B >= 0 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && acap >= 1 && nb >= 1 && C >= 1,
+                  "bad sizes (Hq=%d Hkv=%d acap=%d nb=%d C=%d)", Hq, Hkv, acap, nb, C);
+  FOCUS_CHECK_ARG(aligned16(kbar), "kbar must be 16-byte aligned");
+  if (d != 64 && d != 128) {
+    set_error("head dim %d unsupported (64 or 128)", d);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
+  if (nb > 16384) {
+    set_error("nb=%d exceeds 16384 blocks", nb);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
+  if (B == 0) return FOCUS_OK;
+  const size_t smem = static_cast<size_t>(nb) * sizeof(float);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(Q_active);
+  if (d == 128) {
+    static bool cfg = false;
+    if (!cfg) {
+      cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
+      cfg = true;
+    }
+    block_select_kernel<128><<<B * Hkv, kSelectThreads, smem, s>>>(q, n_active, kbar, Hq, Hkv, acap, nb, C, blocks,
+                                                                     scores_opt);
+  } else {
+    static bool cfg = false;
+    if (!cfg) {
+      cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
+      cfg = true;
+    }
+    block_select_kernel<64><<<B * Hkv, kSelectThreads, smem, s>>>(q, n_active, kbar, Hq, Hkv, acap, nb, C, blocks,
+                                                                    scores_opt);
+  }
+  note_launch();
+  return launch_status("block_select kernel");
+}

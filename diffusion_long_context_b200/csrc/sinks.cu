@@ -1,0 +1,33 @@
+// Attention-sink identification.
+//
+// Focus-dLLM summary page, "核心方法" (core method) and "方法步骤详情" (method steps)
+// step (3): the attention distribution of the dense sink layer, aggregated over the
+// active queries (column sums produced by the dense attention call), picks the sinks;
+// deeper sparse layers reuse them unchanged (cross-layer consistency, abstract).
+// One CTA per (sequence, KV head): block-wide radix top-S over the L column sums.
+#include "focus_common.cuh"
+#include "topk.cuh"
+
+namespace focus {
+
+__global__ void __launch_bounds__(1024) sink_topk_kernel(const float* __restrict__ colsum, int L, int S,
+                                                         int32_t* __restrict__ sinks) {
+  __shared__ TopkShared tk;
+  const int bh = blockIdx.x;
+  const float* row = colsum + static_cast<size_t>(bh) * L;
+  block_topk_ascending([&](int i) { return float_order_key(__ldg(row + i)); }, L, S,
+                       sinks + static_cast<size_t>(bh) * S, S, tk);
+}
+
+}  // namespace focus
+
+using namespace focus;
+
+extern "C" int focus_sink_identify(const float* colsum, int B, int Hkv, int L, int S, int32_t* sinks, void* stream) {
+  FOCUS_CHECK_ARG(colsum && sinks, "null pointer argument");
+  FOCUS_CHECK_ARG(B >= 0 && Hkv >= 1 && L >= 1 && S >= 1 && S <= 4096, "bad sizes (L=%d S=%d)", L, S);
+  if (B == 0) return FOCUS_OK;
+  sink_topk_kernel<<<B * Hkv, 1024, 0, static_cast<cudaStream_t>(stream)>>>(colsum, L, S, sinks);
+  note_launch();
+  return launch_status("sink top-S kernel");
+}

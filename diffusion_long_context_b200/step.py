@@ -1,0 +1,141 @@
+"""The Focus-dLLM denoising step, sequenced over the C-ABI calls.
+
+A non-block-entry step (Focus-dLLM summary page, "方法步骤详情" / method steps (1)-(5)):
+  select_queries -> gather the active query rows of every layer -> layers 0..l_dense:
+  dense attention (layer l_dense also produces the sink column sums) -> sink top-S ->
+  layers > l_dense: block relevance + top-C, sparse attention over sinks U blocks U
+  current block.
+A block-entry step refreshes the block means of every sparse layer (and, for the
+comparison, runs the dense full refresh).
+
+This module only allocates buffers and orders the calls on one CUDA stream; every
+step of the computation runs in libfocus.so kernels. `SparseStep.capture()` records
+the whole step into a CUDA graph so that replay costs one launch from the host.
+"""
+from __future__ import annotations
+
+import math
+from typing import List, Optional
+
+import torch
+
+from . import focus as F
+from .configs import FocusConfig
+
+
+class SparseStep:
+    def __init__(self, cfg: FocusConfig, Q_full: torch.Tensor, K: List[torch.Tensor], V: List[torch.Tensor],
+                 device="cuda"):
+        """Q_full [n_layers, B, Hq, L, d]; K[l], V[l] [B, Hkv, L, d] (bf16, on `device`)."""
+        c = cfg
+        self.cfg = c
+        self.dev = torch.device(device)
+        self.Q_full, self.K, self.V = Q_full, K, V
+        self.scale = 1.0 / math.sqrt(c.d)
+        self.rho = float(torch.tensor(c.rho, dtype=torch.float32))
+        i32 = dict(dtype=torch.int32, device=self.dev)
+        bf = dict(dtype=torch.bfloat16, device=self.dev)
+        self.kcap = max(1, min(c.k, c.G))
+        self.conf_prev = torch.zeros((c.B, c.G), dtype=torch.float32, device=self.dev)
+        self.mask = torch.zeros((c.B, c.L), dtype=torch.uint8, device=self.dev)
+        self.i_focus = torch.full((c.B, self.kcap), -1, **i32)
+        self.n_focus = torch.zeros((c.B,), **i32)
+        self.i_active = torch.full((c.B, c.acap), -1, **i32)
+        self.n_active = torch.zeros((c.B,), **i32)
+        self.Q_active = torch.zeros((c.n_layers, c.B, c.Hq, c.acap, c.d), **bf)
+        self.O_active = torch.zeros((c.n_layers, c.B, c.Hq, c.acap, c.d), **bf)
+        self.colsum = torch.zeros((c.B, c.Hkv, c.L), dtype=torch.float32, device=self.dev)
+        self.sinks = torch.full((c.B, c.Hkv, c.S), -1, **i32)
+        self.sparse_layers = list(range(c.l_dense + 1, c.n_layers))
+        self.kbar = {l: torch.zeros((c.B, c.Hkv, c.nb, c.d), dtype=torch.float32, device=self.dev)
+                     for l in self.sparse_layers}
+        self.blocks = {l: torch.full((c.B, c.Hkv, c.C), -1, **i32) for l in self.sparse_layers}
+        dws = F.dense_workspace_bytes(c.B, c.Hq, c.Hkv, c.L, c.d, c.acap, True)
+        sws = F.sparse_workspace_bytes(c.B, c.Hq, c.Hkv, c.L, c.d, c.acap, c.S, c.C, c.bs, c.P, c.g0, c.g1)
+        self.ws = torch.empty(max(dws, sws, 256), dtype=torch.uint8, device=self.dev)
+        self.graph: Optional[torch.cuda.CUDAGraph] = None
+        self.launches_per_step: Optional[int] = None
+
+    # ------------------------------------------------------------------ inputs
+    def set_state(self, conf_prev: torch.Tensor, mask: torch.Tensor, non_blocking=True):
+        self.conf_prev.copy_(conf_prev, non_blocking=non_blocking)
+        self.mask.copy_(mask, non_blocking=non_blocking)
+
+    # ------------------------------------------------------------------ block entry
+    def block_entry(self):
+        """Block means of every sparse layer (cached for the later steps of the block)."""
+        c = self.cfg
+        for l in self.sparse_layers:
+            F.focus_block_means(self.K[l], c.P, c.bs, self.kbar[l])
+
+    def full_refresh_layer(self, l: int, O_full: torch.Tensor):
+        """Dense full refresh of layer l: every query of the sequence over all L keys."""
+        F.focus_dense_attention(self.Q_full[l], None, self.K[l], self.V[l], O_full, scale=self.scale)
+
+    # ------------------------------------------------------------------ sparse step
+    def select(self):
+        c = self.cfg
+        F.focus_select_queries(self.conf_prev, self.mask, c.g0, c.g1, c.n_t, self.rho, c.w, self.i_focus,
+                               self.n_focus, self.i_active, self.n_active)
+        F.focus_gather_rows(self.Q_full, self.i_active, self.n_active, self.Q_active)
+
+    def dense_layer(self, l: int):
+        c = self.cfg
+        want = l == c.l_dense
+        F.focus_dense_attention(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.O_active[l],
+                                scale=self.scale, colsum=self.colsum if want else None, ws=self.ws)
+        if want:
+            F.focus_sink_identify(self.colsum, c.S, self.sinks)
+
+    def block_select_layer(self, l: int):
+        F.focus_block_select(self.Q_active[l], self.n_active, self.kbar[l], self.cfg.C, self.blocks[l])
+
+    def sparse_attention_layer(self, l: int):
+        c = self.cfg
+        F.focus_sparse_attention(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.sinks,
+                                 self.blocks[l], c.bs, c.P, c.g0, c.g1, self.O_active[l], scale=self.scale,
+                                 ws=self.ws)
+
+    def run(self, timers=None):
+        """Eager step. `timers` (optional) maps a call kind to a list receiving (start, end) events."""
+        c = self.cfg
+
+        def timed(kind, fn, *args):
+            if timers is None:
+                fn(*args)
+                return
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            fn(*args)
+            e.record()
+            timers.setdefault(kind, []).append((s, e))
+
+        timed("select", self.select)
+        for l in range(min(c.l_dense + 1, c.n_layers)):
+            timed("dense_attention" if l != c.l_dense else "dense_attention_colsum", self.dense_layer, l)
+        for l in self.sparse_layers:
+            timed("block_select", self.block_select_layer, l)
+            timed("sparse_attention", self.sparse_attention_layer, l)
+
+    # ------------------------------------------------------------------ graphs
+    def capture(self):
+        before = F.launch_count()
+        self.run()                      # warm: configures kernels, touches every buffer
+        torch.cuda.synchronize()
+        self.launches_per_step = F.launch_count() - before
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                self.run()
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = g
+        return g
+
+    def replay(self):
+        self.graph.replay()
+
+    def release(self):
+        self.graph = None

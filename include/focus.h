@@ -1,0 +1,179 @@
+/*
+ * focus.h -- C ABI of libfocus.so, the B200 (sm_100a) implementation of the
+ * Focus-dLLM sparse denoising-step attention.
+ *
+ * Source of the operations: "Focus-dLLM: Accelerating Long-Context Diffusion LLM
+ * Inference via Confidence-Guided Context Focusing" (summary page of arXiv
+ * 2602.02159), section "方法步骤详情" (method steps) steps (1)-(5), and section
+ * "核心方法" (core method). At a block-entry step the whole sequence runs dense
+ * attention; at every other step:
+ *   (1) PCGI picks the top-k still-[MASK] positions by the previous step's
+ *       confidence, k = floor(rho * n(t))                     -> focus_select_queries
+ *   (2) each is widened to a window of size w -> I_active     -> focus_select_queries
+ *   (3) the first layers run full attention; the attention distribution of the
+ *       sink layer picks the attention sinks                   -> focus_dense_attention,
+ *                                                                focus_sink_identify
+ *   (4) prompt blocks are represented by their mean key, scored against the
+ *       active queries, and the top-C kept                     -> focus_block_means,
+ *                                                                focus_block_select
+ *   (5) the active queries attend over I_p = sinks U kept blocks U current block
+ *                                                              -> focus_sparse_attention
+ *
+ * Conventions shared by every call:
+ *   - Every pointer is a DEVICE pointer unless stated otherwise. The caller owns all
+ *     memory (tensors and workspace); the library allocates nothing.
+ *   - bf16 tensors are passed as `focus_bf16` (raw IEEE bfloat16 bits).
+ *   - Layouts are dense row-major: K, V [B, Hkv, L, d]; Q [B, Hq, qcap, d];
+ *     query head hq uses KV head hq / (Hq / Hkv).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only
+ *     enqueues work on it and never synchronises the host; counts (n_focus,
+ *     n_active) stay on the device.
+ *   - Every call returns a focus_status. Arguments are validated before any launch;
+ *     an invalid call launches nothing and returns FOCUS_ERR_INVALID_ARG (or
+ *     FOCUS_ERR_UNSUPPORTED / FOCUS_ERR_CAPACITY) with a message in
+ *     focus_last_error(). A failed launch returns FOCUS_ERR_CUDA.
+ *   - Index outputs are sorted ascending; unused tail slots hold -1.
+ *   - Every top-k orders by (score descending, index ascending): ties go to the
+ *     lower index and -0.0 equals +0.0. Scores must be finite.
+ *   - A kernel wait that runs out (2 s) records a code in the device error word
+ *     (read it with focus_device_error) and the kernel returns early; outputs of
+ *     that call are then undefined.
+ */
+#ifndef FOCUS_H_
+#define FOCUS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(FOCUS_BUILD) && defined(__GNUC__)
+#define FOCUS_API __attribute__((visibility("default")))
+#else
+#define FOCUS_API
+#endif
+
+typedef uint16_t focus_bf16;
+
+typedef enum {
+  FOCUS_OK = 0,
+  FOCUS_ERR_INVALID_ARG = -1,
+  FOCUS_ERR_UNSUPPORTED = -2,
+  FOCUS_ERR_CUDA = -3,
+  FOCUS_ERR_CAPACITY = -4,
+  FOCUS_ERR_DEVICE_CHECK = -5
+} focus_status;
+
+/* Human-readable name of a status code. Never NULL. */
+FOCUS_API const char* focus_status_string(int status);
+
+/* Message of the last failing call on this host thread ("" if none). Never NULL. */
+FOCUS_API const char* focus_last_error(void);
+
+/* Number of kernels this library has launched in this process (all threads). */
+FOCUS_API uint64_t focus_launch_count(void);
+
+/* Synchronises the current device, copies the device error word to *code_out (0 = no
+ * error) and clears it. Returns FOCUS_ERR_DEVICE_CHECK if the word was set. */
+FOCUS_API int focus_device_error(int* code_out);
+
+/*
+ * (1)+(2) PCGI and window expansion -- method steps (1) and (2).
+ * conf_prev [B, G] fp32, G = g1 - g0: c_{t-1} of position g0 + j at conf_prev[b, j].
+ * mask [B, L] uint8, nonzero = still [MASK]. Candidates: masked positions of the current
+ * block [g0, g1). k = min(floor(rho * n_t), #candidates); I_focus = the top-k candidates
+ * by conf. Each p in I_focus becomes [p - w/2, p - w/2 + w - 1] clipped to [g0, g1);
+ * I_active = the sorted union.
+ * Outputs: i_focus [B, kcap], n_focus [B], i_active [B, acap], n_active [B] (int32).
+ * Requires 0 <= g0 < g1 <= L, G <= 1024, n_t >= 0, rho >= 0, w >= 1,
+ * kcap >= min(floor(rho*n_t), G), acap >= min(G, kcap * w) (else FOCUS_ERR_CAPACITY).
+ */
+FOCUS_API int focus_select_queries(const float* conf_prev, const uint8_t* mask, int B, int L, int g0, int g1, int n_t,
+                         float rho, int w, int32_t* i_focus, int32_t* n_focus, int kcap, int32_t* i_active,
+                         int32_t* n_active, int acap, void* stream);
+
+/*
+ * Gathers rows of a stack of head-major matrices by per-batch row lists (the queries of
+ * the active positions). X [n_mat, B, H, L, d] -> X_rows [n_mat, B, H, cap, d] with
+ * X_rows[m, b, h, i] = X[m, b, h, rows[b, i]] for i < n_rows[b], zero otherwise.
+ * rows [B, cap] and n_rows [B] int32 (device). Row indices outside [0, L) are written
+ * as zero rows and flagged in the device error word (code 5).
+ */
+FOCUS_API int focus_gather_rows(const focus_bf16* X, const int32_t* rows, const int32_t* n_rows, int n_mat, int B, int H,
+                      int L, int d, int cap, focus_bf16* X_rows, void* stream);
+
+/*
+ * (4a) Block representative keys -- method steps (4): the prompt [0, P) is cut into
+ * nb = ceil(P / bs) contiguous blocks; kbar[b, h, j] = mean of K[b, h, j*bs : min(P,(j+1)*bs)].
+ * K [B, Hkv, L, d] bf16 -> kbar [B, Hkv, nb, d] fp32. Requires 1 <= P <= L, bs >= 1,
+ * d in {64, 128}, K 16-byte aligned.
+ */
+FOCUS_API int focus_block_means(const focus_bf16* K, int B, int Hkv, int L, int d, int P, int bs, float* kbar,
+                      void* stream);
+
+/*
+ * (4b) Block relevance and top-C -- method steps (4).
+ * R[b, h, j] = mean over the n_active[b] active queries and the Hq/Hkv query heads of
+ * KV group h of q . kbar[b, h, j] / sqrt(d) (0 when n_active[b] == 0).
+ * blocks[b, h, :] = the top-min(C, nb) blocks, ascending, -1 tail.
+ * Q_active [B, Hq, acap, d] bf16; n_active [B]; kbar [B, Hkv, nb, d] fp32;
+ * scores_opt: NULL or [B, Hkv, nb] fp32 receiving R. Requires nb <= 16384, C >= 1,
+ * d in {64, 128}.
+ */
+FOCUS_API int focus_block_select(const focus_bf16* Q_active, const int32_t* n_active, const float* kbar, int B, int Hq,
+                       int Hkv, int d, int acap, int nb, int C, int32_t* blocks, float* scores_opt,
+                       void* stream);
+
+/*
+ * (3) Dense bidirectional attention -- method steps (3) and the block-entry full refresh.
+ * For query i < n_q[b] (all qcap rows when n_q == NULL) of head hq:
+ *   O[b, hq, i] = softmax_j(scale * q_i . k_j) V over all L keys (fp32 accumulation).
+ * Rows i >= n_q[b] of O are written as zero.
+ * colsum_opt: NULL, or [B, Hkv, L] fp32 receiving the sink importance
+ *   colsum[b, h, j] = sum over the group's query heads and the valid queries of p_ij
+ *   (requires (Hq/Hkv) * qcap <= 256).
+ * ws/ws_bytes: device workspace of at least focus_dense_workspace_bytes(...) bytes,
+ *   256-byte aligned (may be NULL when that size is 0).
+ * Requires d in {64, 128}, Hq % Hkv == 0, L >= 1, Q/K/V/O 16-byte aligned.
+ */
+FOCUS_API int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K, const focus_bf16* V,
+                          int B, int Hq, int Hkv, int L, int d, int qcap, float scale, focus_bf16* O,
+                          float* colsum_opt, void* ws, size_t ws_bytes, void* stream);
+
+FOCUS_API size_t focus_dense_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int qcap, int want_colsum);
+
+/*
+ * (3) Sink identification -- core method / method steps (3): the attention distribution
+ * of the sink layer, aggregated over the active queries, picks the S sinks per KV head,
+ * reused by every deeper sparse layer. sinks[b, h, :] = top-min(S, L) of colsum[b, h, :],
+ * ascending, -1 tail. colsum [B, Hkv, L] fp32 -> sinks [B, Hkv, S] int32. Requires
+ * 1 <= S <= 4096.
+ */
+FOCUS_API int focus_sink_identify(const float* colsum, int B, int Hkv, int L, int S, int32_t* sinks, void* stream);
+
+/*
+ * (5) Sparse attention -- method steps (5): for each active query (i < n_active[b]) of
+ * head hq (KV head h): O_active[b, hq, i] = softmax over I_p of scale * q . k, applied to V,
+ * with I_p = sinks[b, h, :] U (blocks [j*bs, min(P, (j+1)*bs)) for j in blocks[b, h, :])
+ * U [g0, g1) taken as a SET (a key named twice counts once). Negative entries of
+ * sinks/blocks are ignored; entries must otherwise lie in [0, L) and [0, nb). Rows
+ * i >= n_active[b] of O_active are written as zero.
+ * ws/ws_bytes: at least focus_sparse_workspace_bytes(...) bytes, 256-byte aligned.
+ * Requires d in {64, 128}, 0 <= P <= g0 < g1 <= L, bs >= 1, 0 <= S <= 4096,
+ * 1 <= C <= 4096, blocks sorted ascending among their valid entries.
+ */
+FOCUS_API int focus_sparse_attention(const focus_bf16* Q_active, const int32_t* n_active, const focus_bf16* K,
+                           const focus_bf16* V, const int32_t* sinks, int S, const int32_t* blocks, int C, int bs,
+                           int P, int g0, int g1, int B, int Hq, int Hkv, int L, int d, int acap, float scale,
+                           focus_bf16* O_active, void* ws, size_t ws_bytes, void* stream);
+
+FOCUS_API size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int acap, int S, int C, int bs, int P,
+                                    int g0, int g1);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOCUS_H_ */

@@ -1,0 +1,381 @@
+"""GPU parity: every C-ABI call against the fp64 oracle on the same seeded inputs.
+
+Index sets must match exactly; attention outputs within max-abs 2e-2 / mean-abs 2e-3;
+block means within 1e-3 relative. Sizes span several 128-key tiles with ragged tails,
+both head dims, MHA and GQA, and the degenerate cases of the method.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from diffusion_long_context_b200 import configs, inputs
+from oracle import focus_oracle as orc
+from parity_utils import (KBAR_REL, assert_attention_close, assert_tail_is_minus_one, idx_rows)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def F():
+    from diffusion_long_context_b200 import build
+    build.build()
+    from diffusion_long_context_b200 import focus
+    assert torch.cuda.is_available(), "GPU tests need CUDA"
+    return focus
+
+
+def _i32(shape, fill=-7):
+    return torch.full(shape, fill, dtype=torch.int32, device=DEV)
+
+
+def _topk_matches(got, scores, k, rel=1e-4):
+    """Exact top-k match, or a mismatch confined to scores tied within `rel` of the k-th."""
+    exp = orc.top_k_ascending(scores, k).tolist()
+    if got == exp:
+        return True
+    s = np.asarray(scores, dtype=np.float64)
+    kth = np.sort(s)[::-1][min(k, s.size) - 1]
+    tol = rel * max(1.0, abs(kth))
+    diff = set(got) ^ set(exp)
+    assert len(got) == len(exp), f"top-k size {len(got)} != {len(exp)}"
+    assert all(abs(s[i] - kth) <= tol for i in diff), f"top-k mismatch beyond a near-tie: {sorted(diff)}"
+    return False
+
+
+# ------------------------------------------------------------------ select_queries
+def _run_select(F, conf, mask, g0, g1, n_t, rho, w, kcap, acap):
+    B = mask.shape[0]
+    conf_d = torch.from_numpy(conf).to(DEV)
+    mask_d = torch.from_numpy(mask).to(DEV)
+    i_focus, n_focus = _i32((B, kcap)), _i32((B,))
+    i_active, n_active = _i32((B, acap)), _i32((B,))
+    F.focus_select_queries(conf_d, mask_d, g0, g1, n_t, rho, w, i_focus, n_focus, i_active, n_active)
+    torch.cuda.synchronize()
+    return i_focus, n_focus, i_active, n_active
+
+
+def test_select_queries_tiny_config(F):
+    cfg = configs.TINY
+    st = inputs.step_state(cfg)
+    rho = float(np.float32(cfg.rho))
+    i_focus, n_focus, i_active, n_active = _run_select(F, st.conf_prev, st.mask, cfg.g0, cfg.g1, cfg.n_t, rho,
+                                                       cfg.w, cfg.G, cfg.G)
+    ef, ea = orc.select_queries(st.conf_prev, st.mask, cfg.g0, cfg.g1, cfg.n_t, rho, cfg.w)
+    assert idx_rows(i_focus) == [ef[0].tolist()]
+    assert idx_rows(i_active) == [ea[0].tolist()]
+    assert n_focus.tolist() == [len(ef[0])] and n_active.tolist() == [len(ea[0])]
+    assert len(ef[0]) == min(cfg.k, cfg.n_masked)
+    assert_tail_is_minus_one(i_active, n_active.tolist())
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_select_queries_random_batches(F, seed):
+    rng = np.random.default_rng(100 + seed)
+    for _ in range(6):
+        B = int(rng.integers(1, 65))
+        G = int(rng.choice([1, 3, 8, 31, 32, 33, 64, 200, 1024]))
+        g0 = int(rng.integers(0, 50))
+        g1 = g0 + G
+        L = g1 + int(rng.integers(0, 40))
+        mask = np.zeros((B, L), np.uint8)
+        mask[:, g0:g1] = (rng.random((B, G)) < rng.uniform(0.1, 1.0)).astype(np.uint8)
+        mask[:, g1:] = 1
+        vals = np.float32([0.0, -0.0, 0.125, 0.5, 0.5, 0.75, 1.0])
+        conf = np.where(rng.random((B, G)) < 0.5, rng.choice(vals, (B, G)),
+                        rng.random((B, G)).astype(np.float32)).astype(np.float32)
+        n_t = int(rng.integers(0, 9))
+        rho = float(np.float32(rng.choice([1.0, 2.0, 2.5, 4.0, 8.0])))
+        w = int(rng.integers(1, 12))
+        k = min(int(math.floor(rho * n_t)), G)
+        acap = max(1, min(G, k * w))
+        i_focus, n_focus, i_active, n_active = _run_select(F, conf, mask, g0, g1, n_t, rho, w, max(1, k), acap)
+        ef, ea = orc.select_queries(conf, mask, g0, g1, n_t, rho, w)
+        assert idx_rows(i_focus) == [e.tolist() for e in ef]
+        assert idx_rows(i_active) == [e.tolist() for e in ea]
+        assert n_focus.tolist() == [len(e) for e in ef]
+        assert n_active.tolist() == [len(e) for e in ea]
+
+
+def test_select_queries_no_masked_positions(F):
+    mask = np.zeros((2, 64), np.uint8)
+    conf = np.ones((2, 16), np.float32)
+    i_focus, n_focus, i_active, n_active = _run_select(F, conf, mask, 40, 56, 4, 4.0, 8, 16, 16)
+    assert n_focus.tolist() == [0, 0] and n_active.tolist() == [0, 0]
+    assert (i_focus == -1).all() and (i_active == -1).all()
+
+
+# ------------------------------------------------------------------ gather_rows
+def test_gather_rows(F):
+    X = inputs.random_bf16((3, 2, 5, 300, 128), seed=5, device=DEV)
+    rows = torch.tensor([[7, 8, 299, 0, -1, -1], [1, 2, 3, 4, 5, 6]], dtype=torch.int32, device=DEV)
+    n = torch.tensor([4, 6], dtype=torch.int32, device=DEV)
+    out = torch.full((3, 2, 5, 6, 128), 9.0, dtype=torch.bfloat16, device=DEV)
+    F.focus_gather_rows(X, rows, n, out)
+    torch.cuda.synchronize()
+    for b, cnt in enumerate([4, 6]):
+        r = rows[b, :cnt].long()
+        assert torch.equal(out[:, b, :, :cnt], X[:, b][:, :, r])
+        assert (out[:, b, :, cnt:] == 0).all()
+    assert F.device_error() == 0
+
+
+# ------------------------------------------------------------------ block means
+@pytest.mark.parametrize("d,P,bs,L", [(64, 448, 32, 512), (128, 1000, 64, 1100), (128, 333, 128, 400),
+                                      (128, 64, 1, 64), (64, 250, 24, 260)])
+def test_block_means(F, d, P, bs, L):
+    K = inputs.random_bf16((2, 3, L, d), seed=P + bs, device=DEV)
+    nb = -(-P // bs)
+    kbar = torch.empty((2, 3, nb, d), dtype=torch.float32, device=DEV)
+    F.focus_block_means(K, P, bs, kbar)
+    torch.cuda.synchronize()
+    ref = orc.block_means(inputs.to_f64(K), P, bs)
+    got = kbar.cpu().double().numpy()
+    assert np.all(np.abs(got - ref) <= KBAR_REL * np.abs(ref) + 1e-6)
+
+
+# ------------------------------------------------------------------ block select
+@pytest.mark.parametrize("Hq,Hkv,d,nb,C,acap", [(4, 4, 64, 14, 4, 32), (32, 32, 128, 508, 64, 32),
+                                               (28, 4, 128, 252, 32, 32), (8, 2, 128, 1016, 128, 16),
+                                               (4, 4, 128, 7, 16, 32), (2, 1, 64, 3000, 257, 8)])
+def test_block_select(F, Hq, Hkv, d, nb, C, acap):
+    B = 2
+    Q = inputs.random_bf16((B, Hq, acap, d), seed=nb, device=DEV)
+    kbar = inputs.random_f32((B, Hkv, nb, d), seed=nb + 1, device=DEV, lo=-1.0, hi=1.0)
+    n_active = torch.tensor([acap, max(1, acap // 3)], dtype=torch.int32, device=DEV)
+    blocks = _i32((B, Hkv, C))
+    scores = torch.empty((B, Hkv, nb), dtype=torch.float32, device=DEV)
+    F.focus_block_select(Q, n_active, kbar, C, blocks, scores)
+    torch.cuda.synchronize()
+    ref_blocks, R = orc.block_select(inputs.to_f64(Q), n_active.tolist(), inputs.to_f64(kbar), C)
+    np.testing.assert_allclose(scores.cpu().double().numpy(), R, rtol=1e-4, atol=1e-5)
+    got = blocks.cpu().numpy()
+    exact = 0
+    for b in range(B):
+        for h in range(Hkv):
+            g = [int(x) for x in got[b, h] if x >= 0]
+            exact += _topk_matches(g, R[b, h], min(C, nb))
+            assert np.all(got[b, h, min(C, nb):] == -1)
+    assert exact == B * Hkv, f"{B * Hkv - exact} near-tie top-C sets (checked valid)"
+
+
+def test_block_select_empty_active_set(F):
+    Q = inputs.random_bf16((1, 2, 8, 64), seed=1, device=DEV)
+    kbar = inputs.random_f32((1, 2, 10, 64), seed=2, device=DEV)
+    blocks = _i32((1, 2, 3))
+    F.focus_block_select(Q, torch.zeros(1, dtype=torch.int32, device=DEV), kbar, 3, blocks)
+    torch.cuda.synchronize()
+    assert blocks.tolist() == [[[0, 1, 2], [0, 1, 2]]]      # R = 0 everywhere: lowest indices
+
+
+# ------------------------------------------------------------------ sink identify
+@pytest.mark.parametrize("L,S,coarse", [(512, 4, False), (32768, 32, False), (1000, 16, True), (7, 16, True),
+                                        (65536, 300, False)])
+def test_sink_identify(F, L, S, coarse):
+    B, Hkv = 2, 3
+    if coarse:
+        vals = torch.tensor([0.0, -0.0, 0.25, 0.5, 1.0], device=DEV)
+        gen = torch.Generator(device=DEV)
+        gen.manual_seed(L)
+        colsum = vals[torch.randint(0, 5, (B, Hkv, L), generator=gen, device=DEV)].contiguous()
+    else:
+        colsum = inputs.random_f32((B, Hkv, L), seed=L, device=DEV)
+    sinks = _i32((B, Hkv, S))
+    F.focus_sink_identify(colsum, S, sinks)
+    torch.cuda.synchronize()
+    ref = orc.sink_identify(inputs.to_f64(colsum), S)
+    assert np.array_equal(sinks.cpu().numpy(), ref)
+
+
+# ------------------------------------------------------------------ dense attention
+DENSE_CASES = [
+    # B, Hq, Hkv, L, d, qcap, n_q
+    (1, 4, 4, 512, 64, 32, [13]),
+    (2, 4, 4, 1000, 128, 32, [32, 5]),
+    (1, 28, 4, 1500, 128, 32, [29]),
+    (2, 8, 2, 777, 64, 24, [24, 1]),
+    (1, 2, 1, 129, 128, 16, [16]),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,d,qcap,n_q", DENSE_CASES)
+def test_dense_attention_active_with_colsum(F, B, Hq, Hkv, L, d, qcap, n_q):
+    Q = inputs.random_bf16((B, Hq, qcap, d), seed=L, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=L + 1, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=L + 2, device=DEV)
+    nq = torch.tensor(n_q, dtype=torch.int32, device=DEV)
+    O = torch.full((B, Hq, qcap, d), 7.0, dtype=torch.bfloat16, device=DEV)
+    colsum = torch.empty((B, Hkv, L), dtype=torch.float32, device=DEV)
+    scale = 1.0 / math.sqrt(d)
+    F.focus_dense_attention(Q, nq, K, V, O, scale=scale, colsum=colsum)
+    torch.cuda.synchronize()
+    refO, refC, _ = orc.dense_attention(inputs.to_f64(Q), n_q, inputs.to_f64(K), inputs.to_f64(V),
+                                        float(np.float32(scale)), want_colsum=True)
+    assert_attention_close(O, refO, rows_valid=n_q, what="dense attention")
+    np.testing.assert_allclose(colsum.cpu().double().numpy(), refC, rtol=2e-3, atol=1e-6)
+    assert F.device_error() == 0
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,d", [(1, 4, 4, 640, 128), (1, 4, 2, 300, 64), (2, 2, 2, 257, 128)])
+def test_dense_attention_full_refresh(F, B, Hq, Hkv, L, d):
+    Q = inputs.random_bf16((B, Hq, L, d), seed=3 * L, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=3 * L + 1, device=DEV, scale=2.0)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=3 * L + 2, device=DEV)
+    O = torch.empty((B, Hq, L, d), dtype=torch.bfloat16, device=DEV)
+    F.focus_dense_attention(Q, None, K, V, O)
+    torch.cuda.synchronize()
+    refO, _, _ = orc.dense_attention(inputs.to_f64(Q), None, inputs.to_f64(K), inputs.to_f64(V),
+                                     float(np.float32(1.0 / math.sqrt(d))))
+    assert_attention_close(O, refO, what="full refresh")
+
+
+def test_dense_attention_planted_sinks_recovered(F):
+    cfg = configs.TINY
+    st = inputs.step_state(cfg)
+    Qf, K, V = inputs.make_layer(cfg, 0, DEV, st.sink_pos)
+    ef, ea = orc.select_queries(st.conf_prev, st.mask, cfg.g0, cfg.g1, cfg.n_t, cfg.rho, cfg.w)
+    rows = torch.full((1, cfg.acap), -1, dtype=torch.int32, device=DEV)
+    rows[0, :len(ea[0])] = torch.tensor(ea[0], dtype=torch.int32)
+    n = torch.tensor([len(ea[0])], dtype=torch.int32, device=DEV)
+    Qa = torch.empty((1, cfg.Hq, cfg.acap, cfg.d), dtype=torch.bfloat16, device=DEV)
+    F.focus_gather_rows(Qf, rows, n, Qa)
+    O = torch.empty_like(Qa)
+    colsum = torch.empty((1, cfg.Hkv, cfg.L), dtype=torch.float32, device=DEV)
+    F.focus_dense_attention(Qa, n, K, V, O, colsum=colsum)
+    sinks = _i32((1, cfg.Hkv, cfg.S))
+    F.focus_sink_identify(colsum, cfg.S, sinks)
+    torch.cuda.synchronize()
+    _, refC, _ = orc.dense_attention(orc.gather_rows(inputs.to_f64(Qf), ea, cfg.acap), [len(ea[0])],
+                                     inputs.to_f64(K), inputs.to_f64(V), 1 / math.sqrt(cfg.d), True)
+    for h in range(cfg.Hkv):
+        got = [int(x) for x in sinks[0, h].tolist() if x >= 0]
+        assert set(st.sink_pos.tolist()) <= set(got)
+        _topk_matches(got, refC[0, h], cfg.S)
+
+
+# ------------------------------------------------------------------ sparse attention
+SPARSE_CASES = [
+    # name, B, Hq, Hkv, d, P, G, L, bs, C, S, acap, n_active
+    ("tiny", 1, 4, 4, 64, 448, 32, 512, 32, 4, 4, 32, [21]),
+    ("mha_bs64", 2, 4, 4, 128, 1984, 32, 2048, 64, 8, 8, 32, [32, 17]),
+    ("gqa", 1, 28, 4, 128, 2048, 32, 2112, 64, 6, 16, 32, [30]),
+    ("bs128_allblocks", 1, 2, 2, 128, 1024, 32, 1088, 128, 16, 4, 32, [9]),
+    ("bs32_many", 1, 2, 1, 128, 4096, 32, 4160, 32, 64, 32, 32, [32]),
+    ("ragged_bs24", 1, 4, 2, 64, 250, 20, 300, 24, 5, 7, 20, [20]),
+    ("no_sinks", 1, 2, 2, 128, 512, 32, 544, 64, 3, 0, 32, [11]),
+]
+
+
+def _sparse_indices(rng, B, Hkv, P, g0, g1, L, bs, C, S, dup=True):
+    nb = -(-P // bs)
+    blocks = np.full((B, Hkv, C), -1, np.int32)
+    sinks = np.full((B, Hkv, max(S, 1)), -1, np.int32)
+    for b in range(B):
+        for h in range(Hkv):
+            kb = np.sort(rng.choice(nb, size=min(C, nb), replace=False))
+            blocks[b, h, :kb.size] = kb
+            if S:
+                pool = list(range(L))
+                s = set(rng.choice(pool, size=S, replace=False).tolist())
+                if dup and kb.size:
+                    s.pop()
+                    s.add(int(kb[0]) * bs)        # a sink inside a kept block
+                if dup and S > 2:
+                    s.pop()
+                    s.add(g0 + 1)                 # a sink inside the current block
+                sv = np.sort(np.array(sorted(s)))[:S]
+                sinks[b, h, :sv.size] = sv
+    return blocks, (sinks if S else None)
+
+
+@pytest.mark.parametrize("case", SPARSE_CASES, ids=[c[0] for c in SPARSE_CASES])
+def test_sparse_attention(F, case):
+    name, B, Hq, Hkv, d, P, G, L, bs, C, S, acap, n_act = case
+    g0, g1 = P, P + G
+    rng = np.random.default_rng(len(name) * 1000 + L)
+    blocks, sinks = _sparse_indices(rng, B, Hkv, P, g0, g1, L, bs, C, S)
+    Q = inputs.random_bf16((B, Hq, acap, d), seed=L + 11, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=L + 12, device=DEV, scale=1.5)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=L + 13, device=DEV)
+    O = torch.full((B, Hq, acap, d), 3.0, dtype=torch.bfloat16, device=DEV)
+    n_active = torch.tensor(n_act, dtype=torch.int32, device=DEV)
+    blocks_d = torch.from_numpy(blocks).to(DEV)
+    sinks_d = None if sinks is None else torch.from_numpy(sinks).to(DEV)
+    scale = 1.0 / math.sqrt(d)
+    F.focus_sparse_attention(Q, n_active, K, V, sinks_d, blocks_d, bs, P, g0, g1, O, scale=scale)
+    torch.cuda.synchronize()
+    sinks_o = np.full((B, Hkv, 1), -1) if sinks is None else sinks
+    ref = orc.sparse_attention(inputs.to_f64(Q), n_act, inputs.to_f64(K), inputs.to_f64(V), sinks_o, blocks, bs,
+                               P, g0, g1, float(np.float32(scale)))
+    assert_attention_close(O, ref, rows_valid=n_act, what=f"sparse attention ({name})")
+    assert F.device_error() == 0
+
+
+def test_sparse_equals_dense_when_everything_is_kept(F):
+    B, Hq, Hkv, d, bs, G = 1, 4, 2, 128, 64, 32
+    P = 1024
+    g0, g1 = P, P + G
+    L = g1 + 64
+    Q = inputs.random_bf16((B, Hq, 32, d), seed=1, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=2, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=3, device=DEV)
+    n = torch.tensor([32], dtype=torch.int32, device=DEV)
+    blocks = torch.arange(P // bs, dtype=torch.int32, device=DEV).repeat(B, Hkv, 1).contiguous()
+    sinks = torch.arange(g1, L, dtype=torch.int32, device=DEV).repeat(B, Hkv, 1).contiguous()
+    Os = torch.empty((B, Hq, 32, d), dtype=torch.bfloat16, device=DEV)
+    Od = torch.empty_like(Os)
+    F.focus_sparse_attention(Q, n, K, V, sinks, blocks, bs, P, g0, g1, Os)
+    F.focus_dense_attention(Q, n, K, V, Od)
+    torch.cuda.synchronize()
+    assert (Os.float() - Od.float()).abs().max().item() <= 1e-2
+
+
+# ------------------------------------------------------------------ composed step
+def test_composed_step_small(F):
+    """Select -> dense layers (+ sinks) -> block means/select -> sparse layers, vs the oracle."""
+    cfg = configs.scaled(configs.LLADA_8K, 1024, n_layers=4, Hq=4, Hkv=4, l_dense=1, C=4, S=8)
+    st = inputs.step_state(cfg)
+    layers = [inputs.make_layer(cfg, l, DEV, st.sink_pos) for l in range(cfg.n_layers)]
+    rho = float(np.float32(cfg.rho))
+    conf = torch.from_numpy(st.conf_prev).to(DEV)
+    mask = torch.from_numpy(st.mask).to(DEV)
+    i_focus, n_focus = _i32((cfg.B, cfg.G)), _i32((cfg.B,))
+    i_active, n_active = _i32((cfg.B, cfg.acap)), _i32((cfg.B,))
+    F.focus_select_queries(conf, mask, cfg.g0, cfg.g1, cfg.n_t, rho, cfg.w, i_focus, n_focus, i_active, n_active)
+    colsum = torch.empty((cfg.B, cfg.Hkv, cfg.L), dtype=torch.float32, device=DEV)
+    sinks = _i32((cfg.B, cfg.Hkv, cfg.S))
+    outs, blocks_all = {}, {}
+    for l, (Qf, K, V) in enumerate(layers):
+        Qa = torch.empty((cfg.B, cfg.Hq, cfg.acap, cfg.d), dtype=torch.bfloat16, device=DEV)
+        F.focus_gather_rows(Qf, i_active, n_active, Qa)
+        O = torch.empty_like(Qa)
+        if l <= cfg.l_dense:
+            F.focus_dense_attention(Qa, n_active, K, V, O, colsum=colsum if l == cfg.l_dense else None)
+            if l == cfg.l_dense:
+                F.focus_sink_identify(colsum, cfg.S, sinks)
+        else:
+            kbar = torch.empty((cfg.B, cfg.Hkv, cfg.nb, cfg.d), dtype=torch.float32, device=DEV)
+            F.focus_block_means(K, cfg.P, cfg.bs, kbar)
+            blocks = _i32((cfg.B, cfg.Hkv, cfg.C))
+            F.focus_block_select(Qa, n_active, kbar, cfg.C, blocks)
+            F.focus_sparse_attention(Qa, n_active, K, V, sinks, blocks, cfg.bs, cfg.P, cfg.g0, cfg.g1, O)
+            blocks_all[l] = blocks
+        outs[l] = O
+    torch.cuda.synchronize()
+    f64 = [tuple(inputs.to_f64(t) for t in lay) for lay in layers]
+    ref = orc.sparse_step(lambda l: f64[l], cfg.n_layers, cfg.l_dense, st.conf_prev, st.mask, cfg.g0, cfg.g1,
+                          cfg.n_t, rho, cfg.w, cfg.P, cfg.bs, cfg.C, cfg.S, cfg.acap,
+                          float(np.float32(1 / math.sqrt(cfg.d))))
+    assert idx_rows(i_focus) == [a.tolist() for a in ref["I_focus"]]
+    assert idx_rows(i_active) == [a.tolist() for a in ref["I_active"]]
+    for h in range(cfg.Hkv):
+        _topk_matches([int(x) for x in sinks[0, h].tolist() if x >= 0], ref["colsum"][0, h], cfg.S)
+    assert np.array_equal(sinks.cpu().numpy(), ref["sinks"]), "sink sets differ"
+    nA = [len(a) for a in ref["I_active"]]
+    for l in range(cfg.n_layers):
+        if l in blocks_all:
+            assert np.array_equal(blocks_all[l].cpu().numpy(), ref["blocks"][l]), f"layer {l} blocks differ"
+        assert_attention_close(outs[l], ref["O"][l], rows_valid=nA, what=f"layer {l}")
+    assert F.device_error() == 0
