@@ -347,6 +347,6 @@ def test_sparse_duplicates_count_once_and_match_masked_sdpa():
 
 
 def test_sparse_partial_last_block():
-    """P % bs != 0: the last block covers only the valid prompt rows."""
-    Ip = orc.sparse_key_set(np.array([-1]), np.array([2]), 8, 20, 20, 24)
-    assert Ip.tolist() == [16, 17, 18, 19, 20, 21, 22, 23]
+    """P % bs != 0: the last block covers only the valid prompt rows [16, 20), not [16, 24)."""
+    Ip = orc.sparse_key_set(np.array([-1]), np.array([2]), 8, 20, 28, 32)
+    assert Ip.tolist() == [16, 17, 18, 19, 28, 29, 30, 31]
