@@ -61,7 +61,7 @@ class ClockSampler:
         "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
     }
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, local_index: int, period_s: float = 0.005):
         self.ok = False
         self.samples, self.reasons = [], set()
         self.period = period_s
@@ -69,7 +69,13 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            vis = [v.strip() for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+            if vis and local_index < len(vis):
+                ident = vis[local_index]
+                self.h = (pynvml.nvmlDeviceGetHandleByIndex(int(ident)) if ident.isdigit()
+                          else pynvml.nvmlDeviceGetHandleByUUID(ident))
+            else:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(local_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
@@ -271,7 +277,7 @@ def run_ours(args):
             torch.distributed.barrier(device_ids=[local])
         torch.cuda.synchronize()
 
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    sampler = ClockSampler(local)
     with sampler:
         t_pre = time.perf_counter()
         while time.perf_counter() - t_pre < 0.3:

@@ -78,6 +78,11 @@ struct AttnSmem {
   static constexpr uint32_t kBytes = kBook + sizeof(AttnBook) + 1024;  // + alignment slack
 };
 
+// Packed query row held by TMEM lane / A-operand row `lane`. Rows are spread across the
+// four 32-lane quadrants (row j -> lane (j % 4) * 32 + j / 4) so that a partly filled tile
+// (32 active queries of an MHA head) keeps all four softmax warps busy.
+__device__ __forceinline__ int lane_to_row(int lane) { return (lane & 31) * 4 + (lane >> 5); }
+
 __device__ __forceinline__ bool wait_drain(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Q rows -> SWIZZLE_128B K-major tile; P tile cleared once.
   for (int idx = threadIdx.x; idx < kBM * CH; idx += kThreads) {
     const int r = idx / CH, c = idx % CH;
-    const int R = mtile * kBM + r;
+    const int R = mtile * kBM + lane_to_row(r);
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (R < rows_total) {
       const int hq = kvh * a.g + R / a.qcap, i = R % a.qcap;
@@ -339,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax warps 0..3
-    const int r = threadIdx.x;                      // query row of the tile == TMEM lane
-    const int R = mtile * kBM + r;
+    const int r = threadIdx.x;                      // TMEM lane == row of the A operand
+    const int R = mtile * kBM + lane_to_row(r);
     const int hq = kvh * a.g + (R < rows_total ? R / a.qcap : 0);
     const int qi = R % a.qcap;
     const bool row_exists = R < rows_total;

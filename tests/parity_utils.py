@@ -42,3 +42,31 @@ def assert_tail_is_minus_one(t: torch.Tensor, counts):
     for row, n in zip(a, counts):
         assert np.all(row[n:] == -1), "unused index slots must hold -1"
         assert np.all(np.diff(row[:n]) > 0), "indices must be strictly ascending"
+
+
+def topk_matches(got, scores, k, rel=1e-4):
+    """Exact top-k match (returns True), or a mismatch confined to scores tied within `rel`
+    of the k-th score (returns False after checking the GPU set is a valid top-k)."""
+    from oracle import focus_oracle as orc
+    exp = orc.top_k_ascending(scores, k).tolist()
+    if list(got) == exp:
+        return True
+    s = np.asarray(scores, dtype=np.float64)
+    kth = np.sort(s)[::-1][min(k, s.size) - 1]
+    tol = rel * max(1.0, abs(kth))
+    diff = set(got) ^ set(exp)
+    assert len(got) == len(exp), f"top-k size {len(got)} != {len(exp)}"
+    assert all(abs(s[i] - kth) <= tol for i in diff), f"top-k mismatch beyond a near-tie: {sorted(diff)}"
+    return False
+
+
+def assert_index_sets(got_t, scores, k, what):
+    """Per-(b, h) top-k sets of a device tensor [B, H, cap] vs oracle scores [B, H, n]."""
+    got = got_t.detach().to("cpu").numpy()
+    ties = 0
+    for b in range(got.shape[0]):
+        for h in range(got.shape[1]):
+            row = [int(x) for x in got[b, h] if x >= 0]
+            ties += not topk_matches(row, scores[b, h], k)
+            assert np.all(got[b, h, min(k, scores.shape[-1]):] == -1), f"{what}: tail must be -1"
+    return ties

@@ -1,0 +1,143 @@
+"""GPU parity at the workloads' full sizes (8K, 16K GQA, 32K, 32K x 4 sequences).
+
+Each case runs one sink layer (dense attention of the active queries + column sums +
+top-S) and one sparse layer (block means + relevance top-C + sparse attention) of the
+config, in the launch configuration the bench uses, and checks every index set and
+every active-query output row against the fp64 oracle. The full refresh at 32K is
+checked on sampled query rows.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from diffusion_long_context_b200 import configs, inputs
+from oracle import focus_oracle as orc
+from parity_utils import assert_attention_close, assert_index_sets, idx_rows
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def F():
+    from diffusion_long_context_b200 import build
+    build.build()
+    from diffusion_long_context_b200 import focus
+    return focus
+
+
+def _run_two_layers(F, cfg):
+    st = inputs.step_state(cfg)
+    ld = cfg.l_dense
+    lay_d = inputs.make_layer(cfg, ld, DEV, st.sink_pos)
+    lay_s = inputs.make_layer(cfg, ld + 1, DEV, st.sink_pos)
+    i32 = dict(dtype=torch.int32, device=DEV)
+    rho = float(np.float32(cfg.rho))
+    kcap = max(1, min(cfg.k, cfg.G))
+    i_focus, n_focus = torch.empty((cfg.B, kcap), **i32), torch.empty((cfg.B,), **i32)
+    i_active, n_active = torch.empty((cfg.B, cfg.acap), **i32), torch.empty((cfg.B,), **i32)
+    F.focus_select_queries(torch.from_numpy(st.conf_prev).to(DEV), torch.from_numpy(st.mask).to(DEV), cfg.g0,
+                           cfg.g1, cfg.n_t, rho, cfg.w, i_focus, n_focus, i_active, n_active)
+    out = {}
+    for tag, (Qf, K, V) in (("dense", lay_d), ("sparse", lay_s)):
+        Qa = torch.empty((cfg.B, cfg.Hq, cfg.acap, cfg.d), dtype=torch.bfloat16, device=DEV)
+        F.focus_gather_rows(Qf, i_active, n_active, Qa)
+        O = torch.empty_like(Qa)
+        if tag == "dense":
+            colsum = torch.empty((cfg.B, cfg.Hkv, cfg.L), dtype=torch.float32, device=DEV)
+            F.focus_dense_attention(Qa, n_active, K, V, O, colsum=colsum)
+            sinks = torch.empty((cfg.B, cfg.Hkv, cfg.S), **i32)
+            F.focus_sink_identify(colsum, cfg.S, sinks)
+            out.update(colsum=colsum, sinks=sinks)
+        else:
+            kbar = torch.empty((cfg.B, cfg.Hkv, cfg.nb, cfg.d), dtype=torch.float32, device=DEV)
+            F.focus_block_means(K, cfg.P, cfg.bs, kbar)
+            blocks = torch.empty((cfg.B, cfg.Hkv, cfg.C), **i32)
+            F.focus_block_select(Qa, n_active, kbar, cfg.C, blocks)
+            F.focus_sparse_attention(Qa, n_active, K, V, out["sinks"], blocks, cfg.bs, cfg.P, cfg.g0, cfg.g1, O)
+            out.update(kbar=kbar, blocks=blocks)
+        out["O_" + tag] = O
+    torch.cuda.synchronize()
+    assert F.device_error() == 0
+    return st, lay_d, lay_s, i_focus, i_active, out
+
+
+def _oracle_active_rows(Qf, active, cap):
+    """The oracle's own active rows of the generated Q, widened to float64 (no CUDA kernel)."""
+    B, H, _, d = Qf.shape
+    out = np.zeros((B, H, cap, d))
+    for b in range(B):
+        r = torch.as_tensor(active[b], dtype=torch.long, device=Qf.device)
+        out[b, :, :r.numel()] = inputs.to_f64(Qf[b][:, r])
+    return out
+
+
+def _check_against_oracle(cfg, st, lay_d, lay_s, i_focus, i_active, out):
+    rho = float(np.float32(cfg.rho))
+    scale = float(np.float32(1 / math.sqrt(cfg.d)))
+    ef, ea = orc.select_queries(st.conf_prev, st.mask, cfg.g0, cfg.g1, cfg.n_t, rho, cfg.w)
+    assert idx_rows(i_focus) == [e.tolist() for e in ef]
+    assert idx_rows(i_active) == [e.tolist() for e in ea]
+    nA = [a.size for a in ea]
+    assert all(len(f) == min(cfg.k, cfg.n_masked) for f in ef)
+    Kd, Vd = inputs.to_f64(lay_d[1]), inputs.to_f64(lay_d[2])
+    Qa = _oracle_active_rows(lay_d[0], ea, cfg.acap)
+    Od, colsum, _ = orc.dense_attention(Qa, nA, Kd, Vd, scale, want_colsum=True)
+    del Kd, Vd
+    assert_attention_close(out["O_dense"], Od, rows_valid=nA, what=f"{cfg.name} dense layer")
+    np.testing.assert_allclose(out["colsum"].cpu().double().numpy(), colsum, rtol=2e-3, atol=1e-6)
+    sinks = orc.sink_identify(colsum, cfg.S)
+    sink_ties = assert_index_sets(out["sinks"], colsum, cfg.S, f"{cfg.name} sinks")
+    for b in range(cfg.B):
+        for h in range(cfg.Hkv):
+            assert set(st.sink_pos.tolist()) <= set(sinks[b, h].tolist()), "planted sinks not recovered"
+    if sink_ties:
+        # a near-tie picked a different (equally valid) sink: continue with the GPU's sets
+        sinks = out["sinks"].cpu().numpy().astype(np.int64)
+    Ks, Vs = inputs.to_f64(lay_s[1]), inputs.to_f64(lay_s[2])
+    Qa = _oracle_active_rows(lay_s[0], ea, cfg.acap)
+    kbar = orc.block_means(Ks, cfg.P, cfg.bs)
+    got_kbar = out["kbar"].cpu().double().numpy()
+    assert np.all(np.abs(got_kbar - kbar) <= 1e-3 * np.abs(kbar) + 1e-6)
+    blocks, R = orc.block_select(Qa, nA, kbar, cfg.C)
+    block_ties = assert_index_sets(out["blocks"], R, min(cfg.C, cfg.nb), f"{cfg.name} blocks")
+    if block_ties:
+        blocks = out["blocks"].cpu().numpy().astype(np.int64)
+    assert sink_ties == 0 and block_ties == 0, \
+        f"{cfg.name}: {sink_ties} sink / {block_ties} block near-tie sets (valid, but not bit-exact)"
+    Os = orc.sparse_attention(Qa, nA, Ks, Vs, sinks, blocks, cfg.bs, cfg.P, cfg.g0, cfg.g1, scale)
+    assert_attention_close(out["O_sparse"], Os, rows_valid=nA, what=f"{cfg.name} sparse layer")
+
+
+@pytest.mark.parametrize("cfg", [configs.LLADA_8K, configs.DREAM_16K, configs.FULL_32K],
+                         ids=["llada_8k", "dream_16k_gqa", "step_32k"])
+def test_full_size_sink_and_sparse_layer(F, cfg):
+    _check_against_oracle(cfg, *_run_two_layers(F, cfg))
+
+
+@pytest.mark.parametrize("bs,C,rho", [(32, 8, 4.0), (64, 32, 2.0), (128, 128, 8.0)])
+def test_sweep_points_batch4_32k(F, bs, C, rho):
+    cfg = configs.SWEEP_BASE.replace(bs=bs, C=C, rho=rho, n_layers=2, l_dense=0)
+    _check_against_oracle(cfg, *_run_two_layers(F, cfg))
+
+
+def test_full_refresh_32k_sampled_rows(F):
+    """Block-entry dense refresh at 32K: all 32768 queries; 96 sampled rows vs the oracle."""
+    cfg = configs.FULL_32K
+    st = inputs.step_state(cfg)
+    Qf, K, V = inputs.make_layer(cfg, 0, DEV, st.sink_pos)
+    O = torch.empty((cfg.B, cfg.Hq, cfg.L, cfg.d), dtype=torch.bfloat16, device=DEV)
+    F.focus_dense_attention(Qf, None, K, V, O)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(77)
+    heads = rng.choice(cfg.Hq, size=3, replace=False)
+    rows = np.sort(rng.choice(cfg.L, size=32, replace=False))
+    scale = float(np.float32(1 / math.sqrt(cfg.d)))
+    ridx = torch.as_tensor(rows, device=DEV)
+    for hq in heads:
+        q = inputs.to_f64(Qf[:, hq:hq + 1, ridx])                  # [1, 1, 32, d]
+        ref, _, _ = orc.dense_attention(q, None, inputs.to_f64(K[:, hq:hq + 1]), inputs.to_f64(V[:, hq:hq + 1]),
+                                        scale)
+        assert_attention_close(O[:, hq:hq + 1, ridx], ref, what=f"refresh head {hq}")

@@ -12,7 +12,8 @@ import torch
 
 from diffusion_long_context_b200 import configs, inputs
 from oracle import focus_oracle as orc
-from parity_utils import (KBAR_REL, assert_attention_close, assert_tail_is_minus_one, idx_rows)
+from parity_utils import (KBAR_REL, assert_attention_close, assert_tail_is_minus_one, idx_rows,
+                          topk_matches)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -29,20 +30,6 @@ def F():
 
 def _i32(shape, fill=-7):
     return torch.full(shape, fill, dtype=torch.int32, device=DEV)
-
-
-def _topk_matches(got, scores, k, rel=1e-4):
-    """Exact top-k match, or a mismatch confined to scores tied within `rel` of the k-th."""
-    exp = orc.top_k_ascending(scores, k).tolist()
-    if got == exp:
-        return True
-    s = np.asarray(scores, dtype=np.float64)
-    kth = np.sort(s)[::-1][min(k, s.size) - 1]
-    tol = rel * max(1.0, abs(kth))
-    diff = set(got) ^ set(exp)
-    assert len(got) == len(exp), f"top-k size {len(got)} != {len(exp)}"
-    assert all(abs(s[i] - kth) <= tol for i in diff), f"top-k mismatch beyond a near-tie: {sorted(diff)}"
-    return False
 
 
 # ------------------------------------------------------------------ select_queries
@@ -156,7 +143,7 @@ def test_block_select(F, Hq, Hkv, d, nb, C, acap):
     for b in range(B):
         for h in range(Hkv):
             g = [int(x) for x in got[b, h] if x >= 0]
-            exact += _topk_matches(g, R[b, h], min(C, nb))
+            exact += topk_matches(g, R[b, h], min(C, nb))
             assert np.all(got[b, h, min(C, nb):] == -1)
     assert exact == B * Hkv, f"{B * Hkv - exact} near-tie top-C sets (checked valid)"
 
@@ -252,7 +239,7 @@ def test_dense_attention_planted_sinks_recovered(F):
     for h in range(cfg.Hkv):
         got = [int(x) for x in sinks[0, h].tolist() if x >= 0]
         assert set(st.sink_pos.tolist()) <= set(got)
-        _topk_matches(got, refC[0, h], cfg.S)
+        topk_matches(got, refC[0, h], cfg.S)
 
 
 # ------------------------------------------------------------------ sparse attention
@@ -371,7 +358,7 @@ def test_composed_step_small(F):
     assert idx_rows(i_focus) == [a.tolist() for a in ref["I_focus"]]
     assert idx_rows(i_active) == [a.tolist() for a in ref["I_active"]]
     for h in range(cfg.Hkv):
-        _topk_matches([int(x) for x in sinks[0, h].tolist() if x >= 0], ref["colsum"][0, h], cfg.S)
+        topk_matches([int(x) for x in sinks[0, h].tolist() if x >= 0], ref["colsum"][0, h], cfg.S)
     assert np.array_equal(sinks.cpu().numpy(), ref["sinks"]), "sink sets differ"
     nA = [len(a) for a in ref["I_active"]]
     for l in range(cfg.n_layers):
