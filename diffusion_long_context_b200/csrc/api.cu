@@ -3,6 +3,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <mutex>
 
 #include "focus_common.cuh"
@@ -30,6 +31,14 @@ void set_error(const char* fmt, ...) {
   va_start(ap, fmt);
   vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
   va_end(ap);
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("FOCUS_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 void note_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }

@@ -95,6 +95,8 @@ template <int D, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const AttnArgs a) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   using SM = AttnSmem<D>;
   constexpr int CH = D / 8;                // 16-byte chunks per row
   constexpr int ATOMS = D / 64;
@@ -522,6 +524,8 @@ template <int D>
 __global__ void attn_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
                                     const int32_t* __restrict__ n_q, int B, int Hq, int qcap, int n_splits,
                                     __nv_bfloat16* __restrict__ O, float* __restrict__ lse_out) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int total = B * Hq * qcap;
@@ -598,6 +602,8 @@ struct ColSmem {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     colsum_kernel(const __grid_constant__ CUtensorMap tmK128, const ColsumArgs a) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   using SM = ColSmem<D>;
   constexpr int CH = D / 8;
   constexpr int ATOMS = D / 64;
@@ -809,8 +815,12 @@ int launch_attention(const AttnArgs& args, const CUtensorMap& mk, const CUtensor
     configured = true;
   }
   dim3 grid(args.n_splits, n_mtiles, args.B * args.Hkv);
-  kern<<<grid, kThreads, SM::kBytes, stream>>>(mk, mv, args);
+  const cudaError_t e = launch_k(kern, grid, dim3(kThreads), SM::kBytes, stream, mk, mv, args);
   note_launch();
+  if (e != cudaSuccess) {
+    set_error("attention launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
   return launch_status(SPARSE ? "sparse attention kernel" : "dense attention kernel");
 }
 
@@ -818,10 +828,15 @@ template <int D>
 int launch_combine(const AttnArgs& a, cudaStream_t stream) {
   const int rows = a.B * a.Hq * a.qcap;
   const int warps = 8;
-  attn_combine_kernel<D><<<(rows + warps - 1) / warps, warps * 32, 0, stream>>>(
-      a.part_o, a.part_lse, a.n_q, a.B, a.Hq, a.qcap, a.n_splits, a.O, a.lse_out);
+  const cudaError_t e = launch_k(attn_combine_kernel<D>, dim3((rows + warps - 1) / warps), dim3(warps * 32), 0,
+                                 stream, a.part_o, a.part_lse, a.n_q, a.B, a.Hq, a.qcap, a.n_splits, a.O,
+                                 a.lse_out);
   note_launch();
-  return launch_status("attention combine kernel");
+  if (e != cudaSuccess) {
+    set_error("combine launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }
 
 template <int D>
@@ -860,9 +875,13 @@ int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat1
     configured = true;
   }
   dim3 grid(chunks, units);
-  kern<<<grid, kThreads, SM::kBytes, stream>>>(mk, c);
+  const cudaError_t e = launch_k(kern, grid, dim3(kThreads), SM::kBytes, stream, mk, c);
   note_launch();
-  return launch_status("sink column-sum kernel");
+  if (e != cudaSuccess) {
+    set_error("colsum launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }
 
 template <int D, bool SPARSE>

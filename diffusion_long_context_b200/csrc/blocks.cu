@@ -15,6 +15,8 @@ namespace focus {
 template <int D>
 __global__ void __launch_bounds__(256) block_means_kernel(const __nv_bfloat16* __restrict__ K, int L, int P, int bs,
                                                           int nb, float* __restrict__ kbar) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   constexpr int CH = D / 8;
   constexpr int RL = 256 / CH;            // rows in flight per pass
   __shared__ float red[RL][D + 4];
@@ -55,6 +57,8 @@ template <int D>
 __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
     const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ n_active, const float* __restrict__ kbar, int Hq,
     int Hkv, int acap, int nb, int C, int32_t* __restrict__ blocks, float* __restrict__ scores) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   constexpr int PARTS = kSelectThreads / D;
   extern __shared__ float s_R[];           // [nb]
   __shared__ float s_part[PARTS][D];
@@ -123,12 +127,15 @@ extern "C" int focus_block_means(const focus_bf16* K, int B, int Hkv, int L, int
   FOCUS_CHECK_ARG(static_cast<long long>(B) * Hkv < 65536, "B*Hkv must be < 65536");
   dim3 grid(nb, B * Hkv);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    block_means_kernel<128><<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(K), L, P, bs, nb, kbar);
-  else
-    block_means_kernel<64><<<grid, 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(K), L, P, bs, nb, kbar);
+  const __nv_bfloat16* k = reinterpret_cast<const __nv_bfloat16*>(K);
+  const cudaError_t e = d == 128 ? launch_k(block_means_kernel<128>, grid, dim3(256), 0, s, k, L, P, bs, nb, kbar)
+                                 : launch_k(block_means_kernel<64>, grid, dim3(256), 0, s, k, L, P, bs, nb, kbar);
   note_launch();
-  return launch_status("block_means kernel");
+  if (e != cudaSuccess) {
+    set_error("block_means launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }
 
 extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_active, const float* kbar, int B,
@@ -150,23 +157,28 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
   const size_t smem = static_cast<size_t>(nb) * sizeof(float);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(Q_active);
+  cudaError_t err;
   if (d == 128) {
     static bool cfg = false;
     if (!cfg) {
       cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
       cfg = true;
     }
-    block_select_kernel<128><<<B * Hkv, kSelectThreads, smem, s>>>(q, n_active, kbar, Hq, Hkv, acap, nb, C, blocks,
-                                                                     scores_opt);
+    err = launch_k(block_select_kernel<128>, dim3(B * Hkv), dim3(kSelectThreads), smem, s, q, n_active, kbar, Hq,
+                   Hkv, acap, nb, C, blocks, scores_opt);
   } else {
     static bool cfg = false;
     if (!cfg) {
       cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
       cfg = true;
     }
-    block_select_kernel<64><<<B * Hkv, kSelectThreads, smem, s>>>(q, n_active, kbar, Hq, Hkv, acap, nb, C, blocks,
-                                                                    scores_opt);
+    err = launch_k(block_select_kernel<64>, dim3(B * Hkv), dim3(kSelectThreads), smem, s, q, n_active, kbar, Hq,
+                   Hkv, acap, nb, C, blocks, scores_opt);
   }
   note_launch();
-  return launch_status("block_select kernel");
+  if (err != cudaSuccess) {
+    set_error("block_select launch: %s", cudaGetErrorString(err));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }

@@ -12,6 +12,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/focus.h"
 
 namespace focus {
@@ -43,6 +45,31 @@ enum DevErr : int {
 
 static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Programmatic dependent launch is on unless FOCUS_PDL=0 is set in the environment.
+bool pdl_enabled();
+
+#if defined(__CUDACC__)
+// Launches `kernel` with programmatic stream serialization: the launch may overlap the
+// tail of the previous kernel on the stream. Every kernel of this library executes
+// griddep_wait() before it reads global memory, so results are ordered as with a plain
+// launch (and transitively so, because each kernel waits for its predecessor).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+#endif
+
 // ------------------------------------------------------------------ device side
 #if defined(__CUDACC__)
 
@@ -56,6 +83,14 @@ __device__ __forceinline__ unsigned long long globaltimer() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+// Wait until the previous kernel on the stream has completed and its writes are visible
+// (no-op when the kernel was not launched as a programmatic dependent).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream begin launching (its griddep_wait still orders it).
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 __device__ __forceinline__ void record_dev_error(int* err, int code) {

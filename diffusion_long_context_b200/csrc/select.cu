@@ -17,6 +17,8 @@ __global__ void select_queries_kernel(const float* __restrict__ conf, const uint
                                       int g0, int G, int k_req, int w, int32_t* __restrict__ i_focus,
                                       int32_t* __restrict__ n_focus, int kcap, int32_t* __restrict__ i_active,
                                       int32_t* __restrict__ n_active, int acap) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   __shared__ float s_conf[1024];
   __shared__ uint8_t s_cand[1024];
   __shared__ uint8_t s_sel[1024];
@@ -66,6 +68,8 @@ __global__ void select_queries_kernel(const float* __restrict__ conf, const uint
 __global__ void gather_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ rows,
                                    const int32_t* __restrict__ n_rows, int B, int H, int L, int chunks, int cap,
                                    long long total, uint4* __restrict__ out, int* dev_err) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= total) return;
   const int c = static_cast<int>(idx % chunks);
@@ -116,10 +120,15 @@ extern "C" int focus_select_queries(const float* conf_prev, const uint8_t* mask,
   }
   if (B == 0) return FOCUS_OK;
   const int threads = ((G + 31) / 32) * 32;
-  select_queries_kernel<<<B, threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      conf_prev, mask, L, g0, G, k_cap_needed, w, i_focus, n_focus, kcap, i_active, n_active, acap);
+  const cudaError_t e = launch_k(select_queries_kernel, dim3(B), dim3(threads), 0, static_cast<cudaStream_t>(stream),
+                                 conf_prev, mask, L, g0, G, k_cap_needed, w, i_focus, n_focus, kcap, i_active,
+                                 n_active, acap);
   note_launch();
-  return launch_status("select_queries kernel");
+  if (e != cudaSuccess) {
+    set_error("select_queries launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }
 
 extern "C" int focus_gather_rows(const focus_bf16* X, const int32_t* rows, const int32_t* n_rows, int n_mat, int B,
@@ -134,9 +143,14 @@ extern "C" int focus_gather_rows(const focus_bf16* X, const int32_t* rows, const
   const int threads = 256;
   const long long blocks = (total + threads - 1) / threads;
   FOCUS_CHECK_ARG(blocks < (1LL << 31), "too large");
-  gather_rows_kernel<<<static_cast<unsigned>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      reinterpret_cast<const uint4*>(X), rows, n_rows, B, H, L, chunks, cap, total, reinterpret_cast<uint4*>(X_rows),
-      device_error_word());
+  const cudaError_t e =
+      launch_k(gather_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+               static_cast<cudaStream_t>(stream), reinterpret_cast<const uint4*>(X), rows, n_rows, B, H, L, chunks,
+               cap, total, reinterpret_cast<uint4*>(X_rows), device_error_word());
   note_launch();
-  return launch_status("gather_rows kernel");
+  if (e != cudaSuccess) {
+    set_error("gather_rows launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }

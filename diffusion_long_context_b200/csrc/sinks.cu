@@ -12,6 +12,8 @@ namespace focus {
 
 __global__ void __launch_bounds__(1024) sink_topk_kernel(const float* __restrict__ colsum, int L, int S,
                                                          int32_t* __restrict__ sinks) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
   __shared__ TopkShared tk;
   const int bh = blockIdx.x;
   const float* row = colsum + static_cast<size_t>(bh) * L;
@@ -27,7 +29,12 @@ extern "C" int focus_sink_identify(const float* colsum, int B, int Hkv, int L, i
   FOCUS_CHECK_ARG(colsum && sinks, "null pointer argument");
   FOCUS_CHECK_ARG(B >= 0 && Hkv >= 1 && L >= 1 && S >= 1 && S <= 4096, "bad sizes (L=%d S=%d)", L, S);
   if (B == 0) return FOCUS_OK;
-  sink_topk_kernel<<<B * Hkv, 1024, 0, static_cast<cudaStream_t>(stream)>>>(colsum, L, S, sinks);
+  const cudaError_t e =
+      launch_k(sink_topk_kernel, dim3(B * Hkv), dim3(1024), 0, static_cast<cudaStream_t>(stream), colsum, L, S, sinks);
   note_launch();
-  return launch_status("sink top-S kernel");
+  if (e != cudaSuccess) {
+    set_error("sink top-S launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }
