@@ -45,6 +45,8 @@ _SIGS = {
     "focus_sparse_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                     _p, _p, _sz, _p]),
     "focus_sparse_workspace_bytes": (_sz, [_i] * 12),
+    "focus_sparse_attention_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                            _i, _f, _p, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)

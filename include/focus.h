@@ -172,6 +172,32 @@ FOCUS_API int focus_sparse_attention(const focus_bf16* Q_active, const int32_t* 
 FOCUS_API size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int acap, int S, int C, int bs, int P,
                                     int g0, int g1);
 
+/*
+ * Allocation-free variant of focus_sparse_attention. The paper has no counterpart: this
+ * entry point exists for callers that cannot call cudaMalloc, e.g. code that runs while a
+ * stream is being captured in a mode that forbids allocation, plugin hosts whose enqueue
+ * path must not allocate, or servers that reserve all device memory up front. It takes the
+ * same arguments minus the workspace and computes the same result.
+ *
+ * Scratch: the split-KV partials live in one library-owned device array of
+ * FOCUS_NOALLOC_SCRATCH_BYTES bytes (a static __device__ array: every GPU that loads the
+ * library holds it until the process exits). A call whose partials would need more
+ * (focus_sparse_workspace_bytes(...) > FOCUS_NOALLOC_SCRATCH_BYTES) returns
+ * FOCUS_ERR_CAPACITY and launches nothing. The call allocates nothing.
+ * The first call on a device looks the array's device address up (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * All calls share the array and it keeps the previous call's contents; every element a
+ * call reads is written earlier by the same call, so nothing has to be cleared. Calls
+ * that overlap on the GPU (e.g. on two streams without ordering) race on the array.
+ */
+#define FOCUS_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+FOCUS_API int focus_sparse_attention_noalloc(const focus_bf16* Q_active, const int32_t* n_active,
+                                             const focus_bf16* K, const focus_bf16* V, const int32_t* sinks, int S,
+                                             const int32_t* blocks, int C, int bs, int P, int g0, int g1, int B,
+                                             int Hq, int Hkv, int L, int d, int acap, float scale,
+                                             focus_bf16* O_active, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
