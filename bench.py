@@ -299,16 +299,44 @@ def run_ours(args):
     value = ws * n_act / (ms_step * 1e-3)
     gpu_launches = step.launches_per_step * args.steps
 
-    # ---- per-call durations (eager steps, CUDA events on the launching stream)
-    timers = {}
-    for _ in range(max(3, min(args.steps, 10))):
-        step.run(timers=timers)
-    torch.cuda.synchronize()
-    call_ms = {k: float(np.mean(_ev_ms(v))) for k, v in timers.items()}
+    # ---- per-call durations: each call kind of the step captured in its own CUDA graph
+    # (one replay = that call for every layer of the step, so layers rotate and no layer's
+    # K/V stays in L2), timed with CUDA events on the replay stream
+    def graph_ms(fns, reps):
+        gs = torch.cuda.Stream()
+        gs.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gs):
+            for f in fns:
+                f()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=gs):
+                for f in fns:
+                    f()
+            for _ in range(2):
+                g.replay()
+            e0_, e1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0_.record(gs)
+            for _ in range(reps):
+                g.replay()
+            e1_.record(gs)
+        torch.cuda.synchronize()
+        ms = e0_.elapsed_time(e1_) / (reps * len(fns))
+        del g
+        return ms
+
+    reps = max(3, min(args.steps, 20))
+    c = cfg
+    call_ms = {
+        "select_and_gather": graph_ms([step.select], reps),
+        "dense_attention": graph_ms([lambda l=l: step.dense_layer(l) for l in range(c.l_dense)], reps),
+        "dense_attention_colsum_sinks": graph_ms([lambda: step.dense_layer(c.l_dense)], reps),
+        "block_select": graph_ms([lambda l=l: step.block_select_layer(l) for l in step.sparse_layers], reps),
+        "sparse_attention": graph_ms([lambda l=l: step.sparse_attention_layer(l) for l in step.sparse_layers], reps),
+    }
 
     # ---- roofline of the dominant call: the sparse attention of one layer
     hbm, tc, tc_sus, peak_kind = _peaks()
-    c = cfg
     ip_sizes = _key_set_sizes(step)
     mean_ip = float(np.mean(list(ip_sizes.values())))            # summed over (b, kv head)
     A = n_act / c.B
@@ -325,18 +353,12 @@ def run_ours(args):
     step_bytes = n_dense * dense_bytes + colsum_bytes + n_sparse * (sparse_bytes + kbar_bytes)
     step_roof_ms = step_bytes / (hbm * 1e9) * 1e3
 
-    # ---- dense comparator on the same active queries of one sparse layer (all L keys)
-    l0 = step.sparse_layers[0]
-    Od = torch.empty_like(step.O_active[l0])
-    ev = []
-    for _ in range(5):
-        s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s_.record()
-        F.focus_dense_attention(step.Q_active[l0], step.n_active, step.K[l0], step.V[l0], Od, ws=step.ws)
-        e_.record()
-        ev.append((s_, e_))
-    torch.cuda.synchronize()
-    dense_cmp_ms = float(np.median(_ev_ms(ev[1:])))
+    # ---- dense comparator: the same kernel on the same active queries of every sparse
+    # layer, over all L keys (graph replay, as above)
+    Od = torch.empty_like(step.O_active[step.sparse_layers[0]])
+    dense_cmp_ms = graph_ms([lambda l=l: F.focus_dense_attention(step.Q_active[l], step.n_active, step.K[l],
+                                                                 step.V[l], Od, ws=step.ws)
+                             for l in step.sparse_layers], reps)
     kept_ratio = mean_ip / (c.B * c.Hkv * c.L)
 
     # ---- full refresh (block entry comparator): one layer, all L queries
@@ -405,7 +427,7 @@ def run_ours(args):
                        "replay": "one CUDA graph per step", "parallelism": f"replicas x{ws}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": None,
-                         "kernel": "focus_sparse_attention (attention + split combine), one layer",
+                         "kernel": "focus_sparse_attention, one layer (CUDA-graph replay of all sparse layers)",
                          "bytes_per_launch": sparse_bytes, "flops_per_launch": sparse_flops,
                          "launch_ms": call_ms["sparse_attention"], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "roofline_ms": step_roof_ms, "frac": step_roof_ms / ms_step},

@@ -28,14 +28,23 @@
 #include <mutex>
 
 #include "focus_common.cuh"
+#include "slots.cuh"
 
 namespace focus {
+
+// decode_attention.cu
+bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C);
+int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                     __nv_bfloat16* O, float* lse_out, const int32_t* sinks, const int32_t* blocks, int S, int C, int bs,
+                     int P, int g0, int g1, bool sparse, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
+                     cudaStream_t stream);
 
 constexpr int kBM = 128;            // query rows per CTA (tcgen05 M)
 constexpr int kBN = 128;            // keys per tile
 constexpr int kStages = 2;          // K/V pipeline depth
 constexpr int kThreads = 192;       // 6 warps
 constexpr int kMaxSinks = 1024;     // sinks per KV head handled by the sparse kernel
+constexpr int kMaxBlocks = 1024;    // kept blocks per KV head handled by the sparse kernel
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 
@@ -52,6 +61,7 @@ struct AttnArgs {
   const int32_t* blocks;  // [B, Hkv, C]
   int B, Hq, Hkv, L, qcap, g;
   int n_splits, tiles_per_split;
+  int box_rows;           // rows per TMA box (divides 128)
   int S, C, bs, P, g0, g1;
   float scale_log2;
   int* dev_err;
@@ -63,7 +73,8 @@ struct __align__(8) AttnBook {
   uint64_t s_full, s_free, p_full, pv_done, drain;
   uint32_t tmem_base;
   int abort_flag;
-  int n_slots, gen_start, sink_start, n_valid_blocks, last_block_size, n_fsinks, pad_bs;
+  SlotLayout sl;
+  int blk[kMaxBlocks];
   int fsinks[kMaxSinks];
 };
 
@@ -134,61 +145,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (SPARSE) {
-    if (warp == 0) {
-      const int32_t* blk = a.blocks + static_cast<size_t>(bh) * a.C;
-      int nvb = 0;
-      for (int i0 = 0; i0 < a.C; i0 += 32) {
-        const int i = i0 + lane;
-        const bool v = (i < a.C) && (blk[i] >= 0);
-        const unsigned m = __ballot_sync(0xffffffffu, v);
-        nvb += __popc(m);
-        if (m != 0xffffffffu) break;   // valid entries come first
-      }
-      int last_size = a.bs;
-      if (nvb > 0) {
-        const int lb = blk[nvb - 1];
-        last_size = min(a.bs, a.P - lb * a.bs);
-      }
-      // de-duplicated sinks: drop -1, out-of-range, current-block, kept-block and repeated keys
-      const int32_t* snk = a.sinks + static_cast<size_t>(bh) * a.S;
-      int nf = 0;
-      int prev_last = -1;
-      for (int i0 = 0; i0 < a.S; i0 += 32) {
-        const int i = i0 + lane;
-        int j = (i < a.S) ? snk[i] : -1;
-        const int jprev = __shfl_up_sync(0xffffffffu, j, 1);
-        const int before = (lane == 0) ? prev_last : jprev;
-        bool keep = (j >= 0) && (j < a.L) && !(j >= a.g0 && j < a.g1) && (j != before);
-        if (keep && j < a.P) {
-          const int jb = j / a.bs;
-          int lo = 0, hi = nvb - 1;
-          while (lo <= hi) {
-            const int mid = (lo + hi) >> 1;
-            const int v = blk[mid];
-            if (v == jb) { keep = false; break; }
-            if (v < jb) lo = mid + 1; else hi = mid - 1;
-          }
-        }
-        const unsigned m = __ballot_sync(0xffffffffu, keep);
-        const int pos = nf + __popc(m & ((1u << lane) - 1u));
-        if (keep && pos < kMaxSinks) bk->fsinks[pos] = j;
-        nf += __popc(m);
-        prev_last = __shfl_sync(0xffffffffu, j, 31);
-      }
-      if (lane == 0) {
-        const int pad_bs = (a.bs + 7) & ~7;
-        const int G = a.g1 - a.g0;
-        bk->pad_bs = pad_bs;
-        bk->n_valid_blocks = nvb;
-        bk->last_block_size = last_size;
-        bk->gen_start = nvb * pad_bs;
-        bk->sink_start = bk->gen_start + ((G + 7) & ~7);
-        bk->n_fsinks = min(nf, kMaxSinks);
-        bk->n_slots = bk->sink_start + bk->n_fsinks;
-      }
-    }
+    if (warp == 0)
+      build_sparse_layout(a.blocks + static_cast<size_t>(bh) * a.C, a.C,
+                          a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs, a.g0,
+                          a.g1, bk->blk, kMaxBlocks, bk->fsinks, kMaxSinks, &bk->sl);
   } else if (threadIdx.x == 0) {
-    bk->n_slots = a.L;
+    bk->sl.n_slots = a.L;
   }
   // Q rows -> SWIZZLE_128B K-major tile; P tile cleared once.
   for (int idx = threadIdx.x; idx < kBM * CH; idx += kThreads) {
@@ -212,7 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bk->tmem_base;
   const uint32_t tS = tmem;          // columns [0, 128): S, fp32
   const uint32_t tO = tmem + 128;    // columns [128, 128 + D): O, fp32
-  const int n_slots = bk->n_slots;
+  const SlotLayout sl = bk->sl;
+  const int n_slots = sl.n_slots;
   const int total_tiles = (n_slots + kBN - 1) / kBN;
   const int t_begin = split * a.tiles_per_split;
   const int t_end = min(total_tiles, t_begin + a.tiles_per_split);
@@ -225,10 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    const int G = a.g1 - a.g0;
+    const int BR = a.box_rows;
+    const int ngroups = kBN / BR;
     const __nv_bfloat16* Kbh = a.K + static_cast<size_t>(bh) * a.L * D;
     const __nv_bfloat16* Vbh = a.V + static_cast<size_t>(bh) * a.L * D;
-    const int32_t* blk = SPARSE ? a.blocks + static_cast<size_t>(bh) * a.C : nullptr;
     int issued = 0;
     for (int it = 0; it < n_it; ++it) {
       const int s = it % kStages;
@@ -240,61 +203,47 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot0 = (t_begin + it) * kBN;
       uint8_t* dK = sK + s * SM::kTile;
       uint8_t* dV = sV + s * SM::kTile;
-      uint32_t tma_groups = 0;   // bit per 8-row group fetched by TMA
-      int key0s[16];
-#pragma unroll
-      for (int grp = 0; grp < 16; ++grp) {
-        const int gs = slot0 + grp * 8;
-        int key0 = -1;
-        if (!SPARSE) {
-          key0 = gs;
-        } else if (gs < bk->gen_start) {
-          const int i = gs / bk->pad_bs;
-          key0 = blk[i] * a.bs + (gs - i * bk->pad_bs);
-        } else if (gs < bk->sink_start) {
-          key0 = a.g0 + (gs - bk->gen_start);
-        }
-        key0s[grp] = key0;
-        if (key0 >= 0) tma_groups |= 1u << grp;
-      }
-      if (SPARSE) {
-        // rows of the sink segment (and slots past the end) by plain loads; zero if no key
-        for (int grp = 0; grp < 16; ++grp) {
-          if (tma_groups & (1u << grp)) continue;
-          for (int idx = lane; idx < 8 * CH; idx += 32) {
-            const int rr = idx / CH, c = idx % CH;
-            const int slot = slot0 + grp * 8 + rr;
-            const int row = grp * 8 + rr;
-            int key = -1;
-            if (slot >= bk->sink_start && slot < n_slots) key = bk->fsinks[slot - bk->sink_start];
-            uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
-            if (key >= 0) {
-              kv = __ldg(reinterpret_cast<const uint4*>(Kbh + static_cast<size_t>(key) * D) + c);
-              vv = __ldg(reinterpret_cast<const uint4*>(Vbh + static_cast<size_t>(key) * D) + c);
-            }
-            *reinterpret_cast<uint4*>(dK + sw128_offset(row, c, kBN)) = kv;
-            *reinterpret_cast<uint4*>(dV + sw128_offset(row, c, kBN)) = vv;
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-      }
       if (lane == 0) {
-        const uint32_t bytes = static_cast<uint32_t>(__popc(tma_groups)) * ATOMS * 2u * 1024u;
-        mbar_arrive_expect_tx(&bk->full[s], bytes);
-        for (int grp = 0; grp < 16; ++grp) {
-          if (!(tma_groups & (1u << grp))) continue;
+        uint32_t tma_groups = 0;
+        for (int grp = 0; grp < ngroups; ++grp)
+          if (group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR) >= 0) ++tma_groups;
+        mbar_expect_tx(&bk->full[s], tma_groups * ATOMS * 2u * static_cast<uint32_t>(BR) * 128u);
+        for (int grp = 0; grp < ngroups; ++grp) {
+          const int key0 = group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR);
+          if (key0 < 0) continue;
 #pragma unroll
           for (int at = 0; at < ATOMS; ++at) {
-            const uint32_t off = at * (kBN * 128) + grp * 1024;
-            tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, key0s[grp], bh);
-            tma_load_3d(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, key0s[grp], bh);
+            const uint32_t off = at * (kBN * 128) + grp * BR * 128;
+            tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, key0, bh);
+            tma_load_3d(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, key0, bh);
           }
         }
       }
+      if (SPARSE) {
+        // sink rows (and slots past the end, zero-filled) by cp.async, 16 bytes per lane
+        bool any_rows = false;
+        for (int grp = 0; grp < ngroups; ++grp) {
+          if (group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR) >= 0) continue;
+          any_rows = true;
+          for (int idx = lane; idx < BR * CH; idx += 32) {
+            const int rr = idx / CH, c = idx % CH;
+            const int row = grp * BR + rr;
+            const int key = sink_slot_key(sl, bk->fsinks, slot0 + row);
+            const uint32_t src_bytes = key >= 0 ? 16u : 0u;
+            const size_t koff = static_cast<size_t>(key >= 0 ? key : 0) * D + c * 8;
+            cp_async16(smem_u32(dK + sw128_offset(row, c, kBN)), Kbh + koff, src_bytes);
+            cp_async16(smem_u32(dV + sw128_offset(row, c, kBN)), Vbh + koff, src_bytes);
+          }
+        }
+        if (any_rows) {
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mbar_arrive(&bk->full[s]);
       __syncwarp();
       ++issued;
-      (void)G;
     }
     // never leave with copies in flight
     if (lane == 0) {
@@ -368,22 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         unsigned vm[4];
         const int slot0 = (t_begin + it) * kBN;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int slot = slot0 + q * 32 + lane;
-          bool v;
-          if (!SPARSE) {
-            v = slot < a.L;
-          } else if (slot < bk->gen_start) {
-            const int i = slot / bk->pad_bs;
-            const int rr = slot - i * bk->pad_bs;
-            v = rr < ((i == bk->n_valid_blocks - 1) ? bk->last_block_size : a.bs);
-          } else if (slot < bk->sink_start) {
-            v = (slot - bk->gen_start) < (a.g1 - a.g0);
-          } else {
-            v = slot < n_slots;
-          }
-          vm[q] = __ballot_sync(0xffffffffu, v);
-        }
+        for (int q = 0; q < 4; ++q)
+          vm[q] = __ballot_sync(0xffffffffu, slot_valid<SPARSE>(sl, a.L, a.bs, a.g1 - a.g0, slot0 + q * 32 + lane));
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t rg[32];
@@ -577,6 +512,7 @@ struct ColsumArgs {
   float* colsum;          // [B, Hkv, L]
   int B, Hq, Hkv, L, qcap, g, n_pad, tmem_cols;
   int tiles_per_cta;
+  int box_rows;           // rows per TMA box (divides 128)
   float scale_log2;
   int* dev_err;
 };
@@ -674,9 +610,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             !mbar_wait(&bk->empty[s], ((it / kColStages) - 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_PRODUCER))
           break;
         mbar_arrive_expect_tx(&bk->full[s], ATOMS * kBN * 128);
-        for (int at = 0; at < ATOMS; ++at)
-          tma_load_3d(smem_u32(sK + s * SM::kTile + at * (kBN * 128)), &tmK128, &bk->full[s], at * 64,
-                      (t_begin + it) * kBN, bh);
+        for (int r0 = 0; r0 < kBN; r0 += a.box_rows)
+          for (int at = 0; at < ATOMS; ++at)
+            tma_load_3d(smem_u32(sK + s * SM::kTile + at * (kBN * 128) + r0 * 128), &tmK128, &bk->full[s], at * 64,
+                        (t_begin + it) * kBN + r0, bh);
         ++issued;
       }
       for (int j = max(0, issued - kColStages); j < issued; ++j)
@@ -779,14 +716,40 @@ int make_kv_map(CUtensorMap* map, const void* base, int BH, int L, int D, int bo
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+int pow2_rows(int x, int cap) {
+  int r = 8;
+  while (r * 2 <= cap && x % (r * 2) == 0) r *= 2;
+  return r;
+}
+
+// Rows per TMA box: whole tiles for contiguous keys; for the sparse slot layout the
+// largest power of two that keeps every box inside one kept block or the current block.
+int box_rows_for(bool sparse, int L, int bs, int G) {
+  int cap = kBN;
+  while (cap > L && cap > 8) cap >>= 1;
+  if (!sparse) return cap;
+  return std::min(pow2_rows((bs + 7) & ~7, cap), pow2_rows((G + 7) & ~7, cap));
+}
+
+
 struct AttnPlan {
+  bool decode;            // few-query swap-AB kernel (decode_attention.cu) serves this call
   int n_mtiles, n_splits, tiles_per_split;
   size_t lse_bytes, part_lse_bytes, part_o_bytes, total;
 };
 
-AttnPlan plan_attention(int B, int Hq, int Hkv, int d, int qcap, int kv_cap, bool want_lse) {
+// Split plan of a call. The decode kernel merges its splits inside a cluster and needs
+// workspace only for the log-sum-exp consumed by the column-sum pass.
+AttnPlan plan_attention(int B, int Hq, int Hkv, int d, int qcap, int kv_cap, bool want_lse, int L, int S, int C) {
   AttnPlan p{};
   const int g = Hq / Hkv;
+  if (decode_supported(d, Hq, Hkv, qcap, L, S, C)) {
+    p.decode = true;
+    p.n_splits = 1;
+    p.lse_bytes = want_lse ? align256(static_cast<size_t>(B) * Hq * qcap * 4) : 0;
+    p.total = p.lse_bytes;
+    return p;
+  }
   p.n_mtiles = (g * qcap + kBM - 1) / kBM;
   const int max_tiles = std::max(1, (kv_cap + kBN - 1) / kBN);
   const long units = static_cast<long>(B) * Hkv * p.n_mtiles;
@@ -844,9 +807,11 @@ int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat1
                   int B, int Hq, int Hkv, int L, int qcap, float scale_log2, cudaStream_t stream) {
   using SM = ColSmem<D>;
   CUtensorMap mk;
-  int st = make_kv_map(&mk, K, B * Hkv, L, D, kBN);
+  const int box_rows = box_rows_for(false, L, 0, 0);
+  int st = make_kv_map(&mk, K, B * Hkv, L, D, box_rows);
   if (st != FOCUS_OK) return st;
   ColsumArgs c{};
+  c.box_rows = box_rows;
   c.Q = Q;
   c.n_q = n_q;
   c.lse2 = lse2;
@@ -886,12 +851,23 @@ int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat1
 
 template <int D, bool SPARSE>
 int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, cudaStream_t stream) {
-  CUtensorMap mk, mv;
-  int st = make_kv_map(&mk, args.K, args.B * args.Hkv, args.L, D, 8);
-  if (st != FOCUS_OK) return st;
-  st = make_kv_map(&mv, args.V, args.B * args.Hkv, args.L, D, 8);
-  if (st != FOCUS_OK) return st;
   uint8_t* w = static_cast<uint8_t*>(ws);
+  if (plan.decode) {
+    float* lse = plan.lse_bytes ? reinterpret_cast<float*>(w) : nullptr;
+    int st = decode_attention(args.Q, args.n_q, args.K, args.V, args.O, lse, args.sinks, args.blocks, args.S, args.C,
+                              args.bs, args.P, args.g0, args.g1, SPARSE, args.B, args.Hq, args.Hkv, args.L, args.qcap,
+                              args.scale_log2, stream);
+    if (st == FOCUS_OK && colsum)
+      st = launch_colsum<D>(args.Q, args.n_q, args.K, lse, colsum, args.B, args.Hq, args.Hkv, args.L, args.qcap,
+                            args.scale_log2, stream);
+    return st;
+  }
+  args.box_rows = box_rows_for(SPARSE, args.L, args.bs, args.g1 - args.g0);
+  CUtensorMap mk, mv;
+  int st = make_kv_map(&mk, args.K, args.B * args.Hkv, args.L, D, args.box_rows);
+  if (st != FOCUS_OK) return st;
+  st = make_kv_map(&mv, args.V, args.B * args.Hkv, args.L, D, args.box_rows);
+  if (st != FOCUS_OK) return st;
   args.lse_out = plan.lse_bytes ? reinterpret_cast<float*>(w) : nullptr;
   args.part_lse = plan.part_lse_bytes ? reinterpret_cast<float*>(w + plan.lse_bytes) : nullptr;
   args.part_o = plan.part_o_bytes ? reinterpret_cast<float*>(w + plan.lse_bytes + plan.part_lse_bytes) : nullptr;
@@ -916,8 +892,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 int check_common(const void* Q, const void* K, const void* V, const void* O, int B, int Hq, int Hkv, int L, int d,
                  int qcap) {
   FOCUS_CHECK_ARG(Q && K && V && O, "null tensor pointer");
-  FOCUS_CHECK_ARG(B >= 0 && Hq >= 1 && Hkv >= 1 && L >= 1 && qcap >= 1, "bad sizes B=%d Hq=%d Hkv=%d L=%d qcap=%d",
-                  B, Hq, Hkv, L, qcap);
+  FOCUS_CHECK_ARG(B >= 0 && Hq >= 1 && Hkv >= 1 && L >= 8 && qcap >= 1,
+                  "bad sizes B=%d Hq=%d Hkv=%d L=%d (>= 8) qcap=%d", B, Hq, Hkv, L, qcap);
   FOCUS_CHECK_ARG(Hq % Hkv == 0, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
   FOCUS_CHECK_ARG(aligned16(Q) && aligned16(K) && aligned16(V) && aligned16(O), "tensors must be 16-byte aligned");
   FOCUS_CHECK_ARG(static_cast<long long>(B) * Hkv <= 2147483647LL && static_cast<long long>(L) * d < (1LL << 31),
@@ -932,7 +908,7 @@ using namespace focus;
 
 extern "C" size_t focus_dense_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int qcap, int want_colsum) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || qcap <= 0 || Hq % Hkv) return 0;
-  return plan_attention(B, Hq, Hkv, d, qcap, L, want_colsum != 0).total;
+  return plan_attention(B, Hq, Hkv, d, qcap, L, want_colsum != 0, L, 0, 0).total;
 }
 
 extern "C" int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K,
@@ -949,7 +925,7 @@ extern "C" int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, co
     return FOCUS_ERR_UNSUPPORTED;
   }
   if (B == 0) return FOCUS_OK;
-  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, qcap, L, colsum_opt != nullptr);
+  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, qcap, L, colsum_opt != nullptr, L, 0, 0);
   FOCUS_CHECK_ARG(ws_bytes >= plan.total && (plan.total == 0 || ws), "workspace too small: need %zu bytes, got %zu",
                   plan.total, ws_bytes);
   FOCUS_CHECK_ARG((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "workspace must be 256-byte aligned");
@@ -977,7 +953,8 @@ extern "C" size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, in
   const int nb = (P + bs - 1) / bs;
   const long kv_cap = static_cast<long>(std::min(C, std::max(nb, 0))) * ((bs + 7) & ~7) + ((g1 - g0 + 7) & ~7) +
                       std::min(S, kMaxSinks);
-  return plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(std::min<long>(kv_cap, 1 << 30)), false).total;
+  return plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(std::min<long>(kv_cap, 1 << 30)), false, L, S, C)
+      .total;
 }
 
 extern "C" int focus_sparse_attention(const focus_bf16* Q_active, const int32_t* n_active, const focus_bf16* K,
@@ -991,7 +968,11 @@ extern "C" int focus_sparse_attention(const focus_bf16* Q_active, const int32_t*
     return FOCUS_ERR_UNSUPPORTED;
   }
   FOCUS_CHECK_ARG(n_active && blocks && (S == 0 || sinks), "null index pointer");
-  FOCUS_CHECK_ARG(bs >= 1 && C >= 1 && C <= 4096 && S >= 0, "bad bs=%d C=%d S=%d", bs, C, S);
+  FOCUS_CHECK_ARG(bs >= 1 && C >= 1 && S >= 0, "bad bs=%d C=%d S=%d", bs, C, S);
+  if (C > kMaxBlocks) {
+    set_error("C=%d exceeds the %d kept blocks per KV head supported", C, kMaxBlocks);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
   FOCUS_CHECK_ARG(0 <= P && P <= g0 && g0 < g1 && g1 <= L, "need 0 <= P <= g0 < g1 <= L (P=%d g0=%d g1=%d L=%d)", P,
                   g0, g1, L);
   if (S > kMaxSinks) {
@@ -1002,7 +983,7 @@ extern "C" int focus_sparse_attention(const focus_bf16* Q_active, const int32_t*
   const int nb = (P + bs - 1) / bs;
   const long kv_cap = static_cast<long>(std::min(C, nb)) * ((bs + 7) & ~7) + ((g1 - g0 + 7) & ~7) + S;
   FOCUS_CHECK_ARG(kv_cap < (1L << 30), "key set too large");
-  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(kv_cap), false);
+  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(kv_cap), false, L, S, C);
   FOCUS_CHECK_ARG(ws_bytes >= plan.total && (plan.total == 0 || ws), "workspace too small: need %zu bytes, got %zu",
                   plan.total, ws_bytes);
   FOCUS_CHECK_ARG((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "workspace must be 256-byte aligned");

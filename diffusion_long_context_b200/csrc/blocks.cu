@@ -90,18 +90,28 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane < LANES) qv = reinterpret_cast<const float4*>(s_qbar)[lane];
   const float* kb = kbar + static_cast<size_t>(bh) * nb * D;
-  for (int j = warp; j < nb; j += kSelectThreads / 32) {
-    float p = 0.f;
-    if (lane < LANES) {
-      const float4 kv = __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D) + lane);
-      p = qv.x * kv.x + qv.y * kv.y + qv.z * kv.z + qv.w * kv.w;
+  // 8 rows of kbar in flight per warp: 16 warps cover 128 blocks per pass
+  constexpr int UNR = 8;
+  constexpr int NW = kSelectThreads / 32;
+  for (int j0 = warp * UNR; j0 < nb; j0 += NW * UNR) {
+    float4 kv[UNR];
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      const int j = j0 + u;
+      kv[u] = (j < nb && lane < LANES) ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D) + lane)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-    if (lane == 0) {
-      const float R = p * inv_sqrt_d;
-      s_R[j] = R;
-      if (scores) scores[static_cast<size_t>(bh) * nb + j] = R;
+    for (int u = 0; u < UNR; ++u) {
+      float p = qv.x * kv[u].x + qv.y * kv[u].y + qv.z * kv[u].z + qv.w * kv[u].w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+      const int j = j0 + u;
+      if (lane == 0 && j < nb) {
+        const float R = p * inv_sqrt_d;
+        s_R[j] = R;
+        if (scores) scores[static_cast<size_t>(bh) * nb + j] = R;
+      }
     }
   }
   __syncthreads();

@@ -1,0 +1,680 @@
+// Few-query ("decode") attention on the sm_100a tensor cores, swap-AB form.
+//
+// Serves the attentions of a Focus-dLLM sparse step, where only the active queries
+// (about 32 per head) attend:
+//   * dense  (method steps (3)): the active queries over all L keys;
+//   * sparse (method steps (5)): the active queries over I_p = sinks U kept prompt
+//     blocks U current block (slot layout in slots.cuh).
+// With so few queries the 128 keys of a tile are the MMA's M dimension and the queries
+// its N dimension:
+//   S^T[key, q] = K_tile . Q^T        (M = 128 keys, N = NQ queries, K = d)   -> TMEM
+//   O^T[dim, q] += V_tile^T . P^T      (M = d = 128, N = NQ, K = 128 keys)    -> TMEM
+// V_tile^T is the V tile read as an MN-major A operand; P (bf16) is written to shared
+// memory query-major. A softmax thread owns one key of the tile (and one dim of O^T).
+// Each query keeps a reference maximum m_q shared by all keys: p = 2^(s - m_q) while every
+// s stays below m_q + 8; a tile that would exceed it (and the first tile) takes the slow
+// path: the exact per-query tile maximum is reduced across the 128 threads, m_q moves up
+// and O^T and the row sums are rescaled. Row sums are per-thread partials reduced once
+// at the end.
+//
+// Split-KV: the CTAs of one (sequence, KV head) form a thread-block cluster, each takes a
+// contiguous share of the key tiles, and the partial results (m, l, O) are merged through
+// distributed shared memory -- no workspace and no second launch.
+//
+// Warps: 0-3 softmax / epilogue, 4 producer (TMA for key runs, cp.async for sink rows),
+// 5 tcgen05.mma issuer and TMEM owner. K/V tiles flow through a STAGES-deep ring.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "focus_common.cuh"
+#include "slots.cuh"
+
+namespace focus {
+
+constexpr int kDecThreads = 192;
+constexpr int kDecD = 128;
+constexpr int kDecMaxBlocks = 512;
+constexpr int kDecMaxSinks = 512;
+constexpr int kDecProducerWarp = 4;
+constexpr int kDecMmaWarp = 5;
+
+struct DecArgs {
+  const __nv_bfloat16* Q;      // [B, Hq, qcap, D]
+  const int32_t* n_q;          // [B] or null
+  const __nv_bfloat16* K;      // [B, Hkv, L, D]
+  const __nv_bfloat16* V;
+  __nv_bfloat16* O;            // [B, Hq, qcap, D]
+  float* lse_out;              // [B, Hq, qcap] log2 domain, or null
+  const int32_t* sinks;        // [B, Hkv, S]
+  const int32_t* blocks;       // [B, Hkv, C]
+  int B, Hq, Hkv, L, qcap, g;
+  int box_rows;                // rows per TMA box (divides 128)
+  int S, C, bs, P, g0, g1;
+  float scale_log2;
+  int* dev_err;
+};
+
+struct __align__(8) DecBook {
+  uint64_t full[4];
+  uint64_t empty[4];
+  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  SlotLayout sl;
+  float mref[64];
+  float alpha[64];
+  float lfin[64];
+  float red[4][64];
+  int blk[kDecMaxBlocks];
+  int sinks[kDecMaxSinks];
+};
+
+template <int NQ, int STAGES>
+struct DecSmem {
+  static constexpr uint32_t kTile = 128 * kDecD * 2;            // 32 KB
+  static constexpr uint32_t kQ = 0;                             // NQ rows x 256 B
+  static constexpr uint32_t kK = ((NQ * kDecD * 2) + 1023) / 1024 * 1024;
+  static constexpr uint32_t kV = kK + STAGES * kTile;
+  static constexpr uint32_t kP = kV + STAGES * kTile;           // 2 x (NQ rows x 128 keys bf16)
+  static constexpr uint32_t kBook = kP + 2 * NQ * 256;
+  static constexpr uint32_t kBytes = kBook + sizeof(DecBook) + 1024;
+  static constexpr uint32_t kTmemCols = (3 * NQ <= 128) ? 128 : 256;
+};
+
+__device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > 500000000ull) return false;
+  }
+  return true;
+}
+
+template <int NQ, int STAGES, bool SPARSE>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    decode_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const DecArgs a) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
+  using SM = DecSmem<NQ, STAGES>;
+  constexpr int D = kDecD;
+  constexpr int CH = D / 8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + SM::kQ;
+  uint8_t* sK = smem + SM::kK;
+  uint8_t* sV = smem + SM::kV;
+  uint8_t* sP = smem + SM::kP;
+  DecBook* bk = reinterpret_cast<DecBook*>(smem + SM::kBook);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int cs = gridDim.x;                    // CTAs per (b, h) == cluster size
+  const int rank = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / a.Hkv, kvh = bh % a.Hkv;
+  const int nq_b = a.n_q ? min(a.n_q[b], a.qcap) : a.qcap;
+  const int n_rows = a.g * a.qcap;             // <= NQ
+  const int G = a.g1 - a.g0;
+
+  // ---------------------------------------------------------------- prologue
+  if (warp == kDecMmaWarp) {
+    tmem_alloc(&bk->tmem_base, SM::kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&bk->full[s], 1);
+      mbar_init(&bk->empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bk->s_full[i], 1);
+      mbar_init(&bk->s_free[i], 4);
+      mbar_init(&bk->p_full[i], 4);
+      mbar_init(&bk->pv_done[i], 1);
+    }
+    mbar_init(&bk->drain, 1);
+    bk->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (SPARSE) {
+    if (warp == 0)
+      build_sparse_layout(a.blocks + static_cast<size_t>(bh) * a.C, a.C,
+                          a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs, a.g0,
+                          a.g1, bk->blk, kDecMaxBlocks, bk->sinks, kDecMaxSinks, &bk->sl);
+  } else if (threadIdx.x == 0) {
+    bk->sl.n_slots = a.L;
+  }
+  // Q rows (query q <-> head kvh*g + q/qcap, position q%qcap) as a K-major SW128 B operand
+  for (int idx = threadIdx.x; idx < NQ * CH; idx += kDecThreads) {
+    const int q = idx / CH, c = idx % CH;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (q < n_rows) {
+      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
+      if (i < nq_b)
+        v = __ldg(reinterpret_cast<const uint4*>(a.Q + ((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D) + c);
+    }
+    *reinterpret_cast<uint4*>(sQ + sw128_offset(q, c, NQ)) = v;
+  }
+  if (threadIdx.x < NQ) {
+    bk->mref[threadIdx.x] = -INFINITY;
+    bk->alpha[threadIdx.x] = 1.f;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = bk->tmem_base;
+  const SlotLayout sl = bk->sl;
+  const int total_tiles = (sl.n_slots + 127) / 128;
+  const int tps = (total_tiles + cs - 1) / cs;
+  const int t_begin = min(total_tiles, rank * tps);
+  const int n_it = max(0, min(total_tiles, t_begin + tps) - t_begin);
+  volatile int* abort_flag = &bk->abort_flag;
+  float lsum[NQ];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) lsum[q] = 0.f;
+
+  if (warp == kDecProducerWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+    const int BR = a.box_rows;
+    const int ngroups = 128 / BR;
+    const __nv_bfloat16* Kbh = a.K + static_cast<size_t>(bh) * a.L * D;
+    const __nv_bfloat16* Vbh = a.V + static_cast<size_t>(bh) * a.L * D;
+    int issued = 0;
+    for (int it = 0; it < n_it; ++it) {
+      const int s = it % STAGES;
+      if (it >= STAGES &&
+          !__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
+                                             DEV_ERR_TIMEOUT_PRODUCER)))
+        break;
+      const int slot0 = (t_begin + it) * 128;
+      uint8_t* dK = sK + s * SM::kTile;
+      uint8_t* dV = sV + s * SM::kTile;
+      // TMA for contiguous runs
+      if (lane == 0) {
+        uint32_t tma_groups = 0;
+        for (int grp = 0; grp < ngroups; ++grp)
+          if (group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR) >= 0) ++tma_groups;
+        mbar_expect_tx(&bk->full[s], tma_groups * 2u * 2u * static_cast<uint32_t>(BR) * 128u);
+        for (int grp = 0; grp < ngroups; ++grp) {
+          const int key0 = group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR);
+          if (key0 < 0) continue;
+#pragma unroll
+          for (int at = 0; at < 2; ++at) {
+            const uint32_t off = at * (128 * 128) + grp * BR * 128;
+            tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, key0, bh);
+            tma_load_3d(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, key0, bh);
+          }
+        }
+      }
+      if (SPARSE) {
+        // sink rows (and rows past the end, zero-filled) by cp.async, 16 bytes per lane
+        bool any_rows = false;
+        for (int grp = 0; grp < ngroups; ++grp) {
+          if (group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR) >= 0) continue;
+          any_rows = true;
+          for (int idx = lane; idx < BR * CH; idx += 32) {
+            const int rr = idx / CH, c = idx % CH;
+            const int row = grp * BR + rr;
+            const int key = sink_slot_key(sl, bk->sinks, slot0 + row);
+            const uint32_t src_bytes = key >= 0 ? 16u : 0u;
+            const size_t koff = static_cast<size_t>(key >= 0 ? key : 0) * D + c * 8;
+            cp_async16(smem_u32(dK + sw128_offset(row, c, 128)), Kbh + koff, src_bytes);
+            cp_async16(smem_u32(dV + sw128_offset(row, c, 128)), Vbh + koff, src_bytes);
+          }
+        }
+        if (any_rows) {
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mbar_arrive(&bk->full[s]);
+      __syncwarp();
+      ++issued;
+    }
+    if (lane == 0)
+      for (int j = max(0, issued - STAGES); j < issued; ++j) dec_wait_drain(&bk->full[j % STAGES], (j / STAGES) & 1);
+    __syncwarp();
+  } else if (warp == kDecMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(128, NQ, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(128, NQ, true, false);
+      const uint32_t q_base = smem_u32(sQ);
+      const uint32_t tO = tmem + 2 * NQ;
+      bool ok = true;
+      auto issue_pv = [&](int j) -> bool {
+        const int pb = j & 1;
+        if (!mbar_wait(&bk->p_full[pb], (j >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(sV + (j % STAGES) * SM::kTile);
+        const uint32_t p_base = smem_u32(sP + pb * (NQ * 256));
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t da = sw128_desc(v_base + ks * 2048, 128 * 128, 1024);
+          const uint64_t db = sw128_desc(p_base + (ks >> 2) * (NQ * 128) + (ks & 3) * 32, 16, 1024);
+          mma_bf16(tO, da, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+        }
+        mma_commit(&bk->pv_done[pb]);
+        mma_commit(&bk->empty[j % STAGES]);
+        return true;
+      };
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it % STAGES, sb = it & 1;
+        if (!mbar_wait(&bk->full[s], (it / STAGES) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
+        if (it >= 2 && !mbar_wait(&bk->s_free[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
+          break;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(sK + s * SM::kTile);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t da = sw128_desc(k_base + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t db = sw128_desc(q_base + (ks >> 2) * (NQ * 128) + (ks & 3) * 32, 16, 1024);
+          mma_bf16(tmem + sb * NQ, da, db, idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&bk->s_full[sb]);
+        if (it > 0) ok = issue_pv(it - 1);
+      }
+      if (ok && n_it > 0 && !*abort_flag) issue_pv(n_it - 1);
+      mma_commit(&bk->drain);
+      dec_wait_drain(&bk->drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax warps 0..3
+    const int t = threadIdx.x;                         // key of the tile == TMEM lane == dim of O^T
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tO = tmem + 2 * NQ;
+    uint64_t qvalid = 0;                               // bit q: query column q is a real query
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+      if (q < n_rows && (q % a.qcap) < nq_b) qvalid |= (1ull << q);
+    // A warp whose wait ran out keeps iterating without waits or tensor-memory access, so
+    // that all four warps execute the same sequence of named-barrier operations.
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int sb = it & 1;
+      if (ok)
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(&bk->s_full[sb], (it >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_SOFTMAX));
+      float sv[NQ];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) sv[q] = 0.f;
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < NQ / 32; ++c) {
+          uint32_t rg[32];
+          tmem_ld32(tmem + lane_addr + sb * NQ + c * 32, rg);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(rg[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bk->s_free[sb]);
+      const bool kv = ok && slot_valid<SPARSE>(sl, a.L, a.bs, G, (t_begin + it) * 128 + t);
+      bool over = false;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        sv[q] = (kv && ((qvalid >> q) & 1ull)) ? sv[q] * a.scale_log2 : -INFINITY;
+        over |= sv[q] > bk->mref[q] + 8.f;
+      }
+      if (bar_red_or(1, 128, over)) {
+        // exact per-query maximum of this tile, then move the references up
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          float m = sv[q];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (lane == 0) bk->red[warp][q] = m;
+        }
+        named_bar_sync(1, 128);
+        if (t < NQ) {
+          const float mt = fmaxf(fmaxf(bk->red[0][t], bk->red[1][t]), fmaxf(bk->red[2][t], bk->red[3][t]));
+          const float mo = bk->mref[t];
+          const float mn = fmaxf(mo, mt);
+          if (mn > mo + 8.f || (mo == -INFINITY && mn > -INFINITY)) {
+            bk->alpha[t] = (mo == -INFINITY) ? 0.f : exp2_approx(mo - mn);
+            bk->mref[t] = mn;
+          } else {
+            bk->alpha[t] = 1.f;
+          }
+        }
+        named_bar_sync(1, 128);
+        bool any_scale = false;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const float al = bk->alpha[q];
+          lsum[q] *= al;
+          any_scale |= al != 1.f;
+        }
+        if (it > 0 && any_scale && ok) {
+          // O^T must hold PV of the previous tile before it is rescaled
+          ok = __all_sync(0xffffffffu, mbar_wait(&bk->pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag,
+                                                 a.dev_err, DEV_ERR_TIMEOUT_SOFTMAX));
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < NQ / 32; ++c) {
+              uint32_t rg[32];
+              tmem_ld32(tO + lane_addr + c * 32, rg);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) rg[j] = __float_as_uint(__uint_as_float(rg[j]) * bk->alpha[c * 32 + j]);
+              tmem_st32(tO + lane_addr + c * 32, rg);
+            }
+            tmem_st_wait();
+          }
+        }
+      }
+      // P^T of this key: p = 2^(s - m_q)
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const float m = bk->mref[q];
+        sv[q] = exp2_approx(sv[q] - (m == -INFINITY ? 0.f : m));
+        lsum[q] += sv[q];
+      }
+      if (it >= 2 && ok)
+        ok = __all_sync(0xffffffffu, mbar_wait(&bk->pv_done[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err,
+                                               DEV_ERR_TIMEOUT_SOFTMAX));
+      if (ok) {
+        uint8_t* pbuf = sP + sb * (NQ * 256);
+        const uint32_t col = static_cast<uint32_t>((t & 7) * 2);
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const __nv_bfloat16 h = __float2bfloat16_rn(sv[q]);
+          *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128_offset(q, t >> 3, NQ) + col) = h;
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bk->p_full[sb]);
+    }
+    if (ok && n_it > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bk->pv_done[(n_it - 1) & 1], ((n_it - 1) >> 1) & 1, abort_flag,
+                                             a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE));
+      tc_fence_after();
+    }
+    // row sums: reduce the per-key partials over the 128 threads
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      float v = lsum[q];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) bk->red[warp][q] = v;
+    }
+    named_bar_sync(1, 128);
+    if (t < NQ) bk->lfin[t] = (bk->red[0][t] + bk->red[1][t]) + (bk->red[2][t] + bk->red[3][t]);
+    named_bar_sync(1, 128);
+    if (!ok) bk->abort_flag = 1;
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  // Query q is finalised by CTA q % cs of the cluster. Every CTA pushes its partial row of
+  // q (m, l and the unnormalised O row) into the owner's receive buffer with DSMEM stores;
+  // two cluster barriers frame the pushes, and the owner merges from its own memory.
+  // Receive buffer (in the V ring, idle once every CTA of the cluster is past the first
+  // barrier): recv_o[q / cs][src][D], recv_ml[q / cs][src][2].
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const bool have_o = (n_it > 0) && !bk->abort_flag;
+  // index (q / cs) * cs + src < NQ + cs <= NQ + 8: (NQ + 8) x D floats fit in the V ring
+  static_assert((NQ + 8) * (D + 2) * 4 <= STAGES * SM::kTile, "receive buffer exceeds the V ring");
+  float* recv_o = reinterpret_cast<float*>(sV);    // [(q / cs) * cs + src][D]
+  float* recv_ml = recv_o + (NQ + 8) * D;          // [(q / cs) * cs + src][2]
+  float ov[NQ];
+  if (warp < 4) {
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+#pragma unroll
+    for (int c = 0; c < NQ / 32; ++c) {
+      uint32_t rg[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) rg[j] = 0u;
+      if (have_o) {
+        tmem_ld32(tmem + 2 * NQ + lane_addr + c * 32, rg);
+        tmem_ld_wait();
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) ov[c * 32 + j] = __uint_as_float(rg[j]);
+    }
+  }
+  if (cs > 1) cluster_sync();        // every CTA of the cluster is done with its rings
+  else __syncthreads();
+  if (warp < 4) {
+    const int t = threadIdx.x;
+    const uint32_t ro_s = smem_u32(recv_o), rml_s = smem_u32(recv_ml);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      if (q >= n_rows) break;
+      const int owner = q % cs, slot = q / cs;
+      const uint32_t off = static_cast<uint32_t>(((slot * cs + rank) * D + t) * 4);
+      if (cs > 1) {
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_addr(ro_s + off, owner)), "f"(ov[q]) : "memory");
+      } else {
+        recv_o[(slot * cs + rank) * D + t] = ov[q];
+      }
+    }
+    if (t < n_rows) {
+      const int q = t, owner = q % cs, slot = q / cs;
+      const uint32_t off = static_cast<uint32_t>(((slot * cs + rank) * 2) * 4);
+      const float mq = bk->mref[q], lq = have_o ? bk->lfin[q] : 0.f;
+      if (cs > 1) {
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_addr(rml_s + off, owner)), "f"(mq) : "memory");
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_addr(rml_s + off + 4, owner)), "f"(lq) : "memory");
+      } else {
+        recv_ml[(slot * cs + rank) * 2] = mq;
+        recv_ml[(slot * cs + rank) * 2 + 1] = lq;
+      }
+    }
+  }
+  if (cs > 1) cluster_sync();        // pushes visible to their owners
+  else __syncthreads();
+  if (warp < 4) {
+    const int t = threadIdx.x;
+    for (int q = rank; q < n_rows; q += cs) {
+      const int slot = q / cs;
+      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
+      const size_t row = (static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i;
+      float o = 0.f, lse = -INFINITY;
+      if (i < nq_b) {
+        float M = -INFINITY;
+        for (int r = 0; r < cs; ++r) {
+          const float lr = recv_ml[(slot * cs + r) * 2 + 1];
+          if (lr > 0.f) M = fmaxf(M, recv_ml[(slot * cs + r) * 2]);
+        }
+        if (M > -INFINITY) {
+          float l = 0.f;
+          for (int r = 0; r < cs; ++r) {
+            const float lr = recv_ml[(slot * cs + r) * 2 + 1];
+            if (!(lr > 0.f)) continue;
+            const float w = exp2_approx(recv_ml[(slot * cs + r) * 2] - M);
+            l += w * lr;
+            o += w * recv_o[(slot * cs + r) * D + t];
+          }
+          o /= l;
+          lse = M + __log2f(l);
+        }
+      }
+      a.O[row * D + t] = __float2bfloat16_rn(o);
+      if (t == 0 && a.lse_out && i < nq_b) a.lse_out[row] = lse;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kDecMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, SM::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------- host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 dec_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int dec_make_map(CUtensorMap* map, const void* base, int BH, int L, int box_rows) {
+  auto fn = dec_encode_fn();
+  if (!fn) {
+    set_error("cuTensorMapEncodeTiled is unavailable (driver entry point lookup failed)");
+    return FOCUS_ERR_CUDA;
+  }
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kDecD), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kDecD) * 2, static_cast<cuuint64_t>(L) * kDecD * 2};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
+}
+
+template <int NQ, int STAGES, bool SPARSE>
+int max_active_clusters(int cs) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  auto key = std::make_pair(dev, cs);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(DecSmem<NQ, STAGES>::kBytes));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, 1, 1);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = DecSmem<NQ, STAGES>::kBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = cs;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache[key] = n;
+  return n;
+}
+
+template <int NQ, int STAGES, bool SPARSE>
+int choose_cluster(int units) {
+  const int sms = device_sm_count();
+  for (int cs : {8, 4, 2}) {
+    if (units * cs > sms) continue;
+    if (max_active_clusters<NQ, STAGES, SPARSE>(cs) >= units) return cs;
+  }
+  return 1;
+}
+
+template <int NQ, int STAGES, bool SPARSE>
+int run_decode(const DecArgs& a0, cudaStream_t stream) {
+  DecArgs a = a0;
+  CUtensorMap mk, mv;
+  int st = dec_make_map(&mk, a.K, a.B * a.Hkv, a.L, a.box_rows);
+  if (st != FOCUS_OK) return st;
+  st = dec_make_map(&mv, a.V, a.B * a.Hkv, a.L, a.box_rows);
+  if (st != FOCUS_OK) return st;
+  a.dev_err = device_error_word();
+  const int units = a.B * a.Hkv;
+  const int cs = choose_cluster<NQ, STAGES, SPARSE>(units);
+  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(DecSmem<NQ, STAGES>::kBytes));
+  const cudaError_t e =
+      launch_k_cluster(kern, dim3(cs, units), dim3(kDecThreads), DecSmem<NQ, STAGES>::kBytes, stream, cs, mk, mv, a);
+  note_launch();
+  if (e != cudaSuccess) {
+    set_error("decode attention launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
+}
+
+int pow2_divisor(int x, int cap) {
+  int r = 8;
+  while (r * 2 <= cap && x % (r * 2) == 0) r *= 2;
+  return r;
+}
+
+}  // namespace
+
+// Whether the decode kernel serves this shape (else the 128-row tile kernel does).
+bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C) {
+  return d == kDecD && (Hq / Hkv) * qcap <= 64 && L >= 8 && S <= kDecMaxSinks && C <= kDecMaxBlocks;
+}
+
+int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                     __nv_bfloat16* O, float* lse_out, const int32_t* sinks, const int32_t* blocks, int S, int C, int bs,
+                     int P, int g0, int g1, bool sparse, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
+                     cudaStream_t stream) {
+  DecArgs a{};
+  a.Q = Q;
+  a.n_q = n_q;
+  a.K = K;
+  a.V = V;
+  a.O = O;
+  a.lse_out = lse_out;
+  a.sinks = sinks;
+  a.blocks = blocks;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.qcap = qcap;
+  a.g = Hq / Hkv;
+  a.S = S;
+  a.C = C;
+  a.bs = bs;
+  a.P = P;
+  a.g0 = g0;
+  a.g1 = g1;
+  a.scale_log2 = scale_log2;
+  int cap = 128;
+  while (cap > L) cap >>= 1;
+  if (sparse) {
+    const int pad_bs = (bs + 7) & ~7, pad_g = (g1 - g0 + 7) & ~7;
+    a.box_rows = std::min(pow2_divisor(pad_bs, cap), pow2_divisor(pad_g, cap));
+  } else {
+    a.box_rows = cap;
+  }
+  const int nrows = a.g * qcap;
+  if (nrows <= 32)
+    return sparse ? run_decode<32, 3, true>(a, stream) : run_decode<32, 3, false>(a, stream);
+  return sparse ? run_decode<64, 2, true>(a, stream) : run_decode<64, 2, false>(a, stream);
+}
+
+}  // namespace focus

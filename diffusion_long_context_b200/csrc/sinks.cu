@@ -10,16 +10,33 @@
 
 namespace focus {
 
+// The L column sums of (b, h) are staged in shared memory when they fit (STAGE = true).
+template <bool STAGE>
 __global__ void __launch_bounds__(1024) sink_topk_kernel(const float* __restrict__ colsum, int L, int S,
                                                          int32_t* __restrict__ sinks) {
   griddep_wait();               // inputs may come from the previous kernel on the stream
   griddep_launch_dependents();
+  extern __shared__ float s_row[];
   __shared__ TopkShared tk;
   const int bh = blockIdx.x;
   const float* row = colsum + static_cast<size_t>(bh) * L;
-  block_topk_ascending([&](int i) { return float_order_key(__ldg(row + i)); }, L, S,
-                       sinks + static_cast<size_t>(bh) * S, S, tk);
+  if (STAGE) {
+    if ((L & 3) == 0) {
+      for (int i = threadIdx.x; i < L / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(s_row)[i] = __ldg(reinterpret_cast<const float4*>(row) + i);
+    } else {
+      for (int i = threadIdx.x; i < L; i += blockDim.x) s_row[i] = __ldg(row + i);
+    }
+    __syncthreads();
+    block_topk_ascending([&](int i) { return float_order_key(s_row[i]); }, L, S,
+                         sinks + static_cast<size_t>(bh) * S, S, tk);
+  } else {
+    block_topk_ascending([&](int i) { return float_order_key(__ldg(row + i)); }, L, S,
+                         sinks + static_cast<size_t>(bh) * S, S, tk);
+  }
 }
+
+constexpr int kSinkStageMaxBytes = 160 * 1024;
 
 }  // namespace focus
 
@@ -29,8 +46,21 @@ extern "C" int focus_sink_identify(const float* colsum, int B, int Hkv, int L, i
   FOCUS_CHECK_ARG(colsum && sinks, "null pointer argument");
   FOCUS_CHECK_ARG(B >= 0 && Hkv >= 1 && L >= 1 && S >= 1 && S <= 4096, "bad sizes (L=%d S=%d)", L, S);
   if (B == 0) return FOCUS_OK;
-  const cudaError_t e =
-      launch_k(sink_topk_kernel, dim3(B * Hkv), dim3(1024), 0, static_cast<cudaStream_t>(stream), colsum, L, S, sinks);
+  const size_t stage_bytes = static_cast<size_t>(L) * sizeof(float);
+  const bool stage = stage_bytes <= kSinkStageMaxBytes && (reinterpret_cast<uintptr_t>(colsum) & 15u) == 0;
+  cudaError_t e;
+  if (stage) {
+    static bool cfg = false;
+    if (!cfg) {
+      cudaFuncSetAttribute(sink_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSinkStageMaxBytes);
+      cfg = true;
+    }
+    e = launch_k(sink_topk_kernel<true>, dim3(B * Hkv), dim3(1024), stage_bytes, static_cast<cudaStream_t>(stream),
+                 colsum, L, S, sinks);
+  } else {
+    e = launch_k(sink_topk_kernel<false>, dim3(B * Hkv), dim3(1024), 0, static_cast<cudaStream_t>(stream), colsum, L,
+                 S, sinks);
+  }
   note_launch();
   if (e != cudaSuccess) {
     set_error("sink top-S launch: %s", cudaGetErrorString(e));

@@ -1,9 +1,14 @@
 // Block-wide top-k selection shared by the block (top-C) and sink (top-S) kernels.
 //
 // Order: larger key first, ties to the lower index. Keys are order-preserving 32-bit
-// images of the scores (float_order_key), so -0.0 and +0.0 tie. An 8-bit radix select
-// (four histogram passes) finds the k-th largest key T; one ordered pass then keeps
-// every key > T and the lowest-index keys == T, writing the indices in ascending order.
+// images of the scores (float_order_key), so -0.0 and +0.0 tie.
+//   1. Radix select, 8 bits per pass (4 passes), finds T = the k-th largest key and how
+//      many keys equal to T are taken. Histograms use warp-aggregated shared atomics
+//      (lanes with the same digit add once), so a digit shared by every key does not
+//      serialise the CTA; one warp locates the digit with a lane-parallel suffix scan.
+//   2. Ordered selection: each warp owns a contiguous segment of indices; a first walk
+//      counts keys > T and == T per warp, one block barrier turns the counts into
+//      offsets, and a second walk writes the selected indices in ascending order.
 #pragma once
 
 #include "focus_common.cuh"
@@ -32,15 +37,18 @@ __device__ __forceinline__ int block_excl_scan(bool flag, int* s_warp, int& tota
 struct TopkShared {
   int hist[256];
   int s_warp[32];
+  int w_gt[32];
+  int w_eq[32];
   uint32_t prefix;
   int remaining;
 };
 
 // key_of(i) -> uint32 key for i in [0, n). Writes out[0 .. min(k, n)) ascending and -1 into
-// out[min(k, n) .. cap). Every thread of the CTA must call it.
+// out[min(k, n) .. cap). Every thread of the CTA (a multiple of 32 threads) must call it.
 template <typename KeyFn>
 __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, int cap, TopkShared& sm) {
   const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
   k = min(k, n);
   if (k <= 0) {
     for (int i = tid; i < cap; i += nt) out[i] = -1;
@@ -54,48 +62,97 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
     sm.prefix = 0u;
     sm.remaining = k;
   }
-  __syncthreads();
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
     for (int i = tid; i < 256; i += nt) sm.hist[i] = 0;
     __syncthreads();
     const uint32_t prefix = sm.prefix;
-    for (int i = tid; i < n; i += nt) {
-      const uint32_t key = key_of(i);
-      if ((key & hi_mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & 255u], 1);
+    for (int base = 0; base < n; base += nt) {
+      const int i = base + tid;
+      uint32_t bin = 256u;                       // no digit: outside the candidate set
+      if (i < n) {
+        const uint32_t key = key_of(i);
+        if ((key & hi_mask) == prefix) bin = (key >> shift) & 255u;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], __popc(peers));
     }
     __syncthreads();
-    if (tid == 0) {
-      int cum = 0, rem = sm.remaining, sel = 0;
-      for (int bin = 255; bin >= 0; --bin) {
-        const int h = sm.hist[bin];
-        if (cum + h >= rem) {
-          sel = bin;
-          break;
-        }
-        cum += h;
+    if (warp == 0) {
+      // lane l owns digits 255-8l .. 248-8l (descending); find the digit holding the
+      // remaining-th largest candidate
+      int c[8], own = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = sm.hist[255 - 8 * lane - j];
+        own += c[j];
       }
-      sm.remaining = rem - cum;
-      sm.prefix = prefix | (static_cast<uint32_t>(sel) << shift);
+      int incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int rem = sm.remaining;
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= rem);
+      const int L = __ffs(hit) - 1;              // always found: the counts add up to >= rem
+      if (lane == L) {
+        int cum = incl - own;
+        int digit = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (cum + c[j] >= rem) {
+            digit = 255 - 8 * lane - j;
+            break;
+          }
+          cum += c[j];
+        }
+        sm.remaining = rem - cum;
+        sm.prefix = prefix | (static_cast<uint32_t>(digit) << shift);
+      }
     }
     __syncthreads();
   }
   const uint32_t T = sm.prefix;
-  const int take_eq = sm.remaining;   // keys equal to T to keep (lowest indices first)
-  int run_eq = 0, run_sel = 0;
-  for (int base = 0; base < n; base += nt) {
-    const int i = base + tid;
-    const uint32_t key = (i < n) ? key_of(i) : 0u;
-    const bool gt = (i < n) && key > T;
-    const bool eq = (i < n) && key == T;
-    int eq_total = 0, sel_total = 0;
-    const int eq_pos = run_eq + block_excl_scan(eq, sm.s_warp, eq_total);
-    const bool sel = gt || (eq && eq_pos < take_eq);
-    const int pos = run_sel + block_excl_scan(sel, sm.s_warp, sel_total);
+  const int take_eq = sm.remaining;              // keys equal to T to keep (lowest indices first)
+  // ordered selection over warp-owned contiguous segments
+  const int seg = ((n + nwarps - 1) / nwarps + 31) & ~31;
+  const int w_begin = min(n, warp * seg), w_end = min(n, w_begin + seg);
+  int gt = 0, eq = 0;
+  for (int base = w_begin; base < w_end; base += 32) {
+    const int i = base + lane;
+    uint32_t key = 0u;
+    if (i < w_end) key = key_of(i);
+    gt += __popc(__ballot_sync(0xffffffffu, i < w_end && key > T));
+    eq += __popc(__ballot_sync(0xffffffffu, i < w_end && key == T));
+  }
+  if (lane == 0) {
+    sm.w_gt[warp] = gt;
+    sm.w_eq[warp] = eq;
+  }
+  __syncthreads();
+  int gt_before = 0, eq_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_before += sm.w_gt[w];
+    eq_before += sm.w_eq[w];
+  }
+  int run_eq = eq_before;
+  int run_sel = gt_before + min(eq_before, take_eq);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = w_begin; base < w_end; base += 32) {
+    const int i = base + lane;
+    uint32_t key = 0u;
+    if (i < w_end) key = key_of(i);
+    const bool is_gt = i < w_end && key > T;
+    const bool is_eq = i < w_end && key == T;
+    const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
+    const bool sel = is_gt || (is_eq && run_eq + __popc(meq & lt) < take_eq);
+    const unsigned msel = __ballot_sync(0xffffffffu, sel);
+    const int pos = run_sel + __popc(msel & lt);
     if (sel && pos < cap) out[pos] = i;
-    run_eq += eq_total;
-    run_sel += sel_total;
+    run_eq += __popc(meq);
+    run_sel += __popc(msel);
   }
   for (int i = k + tid; i < cap; i += nt) out[i] = -1;
 }

@@ -136,7 +136,7 @@ FOCUS_API int focus_block_select(const focus_bf16* Q_active, const int32_t* n_ac
  *   (requires (Hq/Hkv) * qcap <= 256).
  * ws/ws_bytes: device workspace of at least focus_dense_workspace_bytes(...) bytes,
  *   256-byte aligned (may be NULL when that size is 0).
- * Requires d in {64, 128}, Hq % Hkv == 0, L >= 1, Q/K/V/O 16-byte aligned.
+ * Requires d in {64, 128}, Hq % Hkv == 0, L >= 8, Q/K/V/O 16-byte aligned.
  */
 FOCUS_API int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K, const focus_bf16* V,
                           int B, int Hq, int Hkv, int L, int d, int qcap, float scale, focus_bf16* O,
@@ -161,8 +161,8 @@ FOCUS_API int focus_sink_identify(const float* colsum, int B, int Hkv, int L, in
  * sinks/blocks are ignored; entries must otherwise lie in [0, L) and [0, nb). Rows
  * i >= n_active[b] of O_active are written as zero.
  * ws/ws_bytes: at least focus_sparse_workspace_bytes(...) bytes, 256-byte aligned.
- * Requires d in {64, 128}, 0 <= P <= g0 < g1 <= L, bs >= 1, 0 <= S <= 4096,
- * 1 <= C <= 4096, blocks sorted ascending among their valid entries.
+ * Requires d in {64, 128}, L >= 8, 0 <= P <= g0 < g1 <= L, bs >= 1, 0 <= S <= 1024,
+ * 1 <= C <= 1024, blocks sorted ascending among their valid entries.
  */
 FOCUS_API int focus_sparse_attention(const focus_bf16* Q_active, const int32_t* n_active, const focus_bf16* K,
                            const focus_bf16* V, const int32_t* sinks, int S, const int32_t* blocks, int C, int bs,

@@ -184,6 +184,8 @@ DENSE_CASES = [
     (1, 28, 4, 1500, 128, 32, [29]),
     (2, 8, 2, 777, 64, 24, [24, 1]),
     (1, 2, 1, 129, 128, 16, [16]),
+    (1, 8, 4, 700, 128, 32, [27]),          # 2 query heads per KV head x 32: 64 query columns
+    (2, 32, 32, 600, 128, 32, [32, 19]),    # 64 heads: clusters of 2
 ]
 
 
@@ -252,6 +254,9 @@ SPARSE_CASES = [
     ("bs32_many", 1, 2, 1, 128, 4096, 32, 4160, 32, 64, 32, 32, [32]),
     ("ragged_bs24", 1, 4, 2, 64, 250, 20, 300, 24, 5, 7, 20, [20]),
     ("no_sinks", 1, 2, 2, 128, 512, 32, 544, 64, 3, 0, 32, [11]),
+    ("gqa2_nq64", 1, 8, 4, 128, 1024, 32, 1100, 64, 5, 9, 32, [32]),
+    ("mha64_heads", 2, 32, 32, 128, 640, 32, 700, 32, 4, 6, 32, [25, 32]),
+    ("bs16_mha", 1, 4, 4, 128, 512, 32, 560, 16, 12, 5, 32, [30]),
 ]
 
 
