@@ -62,6 +62,7 @@ struct AttnArgs {
   int B, Hq, Hkv, L, qcap, g;
   int n_splits, tiles_per_split;
   int box_rows;           // rows per TMA box (divides 128)
+  int gen_pad;            // slots of the current block in the sparse layout (multiple of box_rows)
   int S, C, bs, P, g0, g1;
   float scale_log2;
   int* dev_err;
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0)
       build_sparse_layout(a.blocks + static_cast<size_t>(bh) * a.C, a.C,
                           a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs, a.g0,
-                          a.g1, bk->blk, kMaxBlocks, bk->fsinks, kMaxSinks, &bk->sl);
+                          a.g1, a.gen_pad, bk->blk, kMaxBlocks, bk->fsinks, kMaxSinks, &bk->sl);
   } else if (threadIdx.x == 0) {
     bk->sl.n_slots = a.L;
   }
@@ -725,11 +726,15 @@ int pow2_rows(int x, int cap) {
 // Rows per TMA box: whole tiles for contiguous keys; for the sparse slot layout the
 // largest power of two that keeps every box inside one kept block or the current block.
 int box_rows_for(bool sparse, int L, int bs, int G) {
+  (void)G;
   int cap = kBN;
   while (cap > L && cap > 8) cap >>= 1;
   if (!sparse) return cap;
-  return std::min(pow2_rows((bs + 7) & ~7, cap), pow2_rows((G + 7) & ~7, cap));
+  return pow2_rows((bs + 7) & ~7, cap);
 }
+
+// The current block is padded to whole boxes so that every box stays in one segment.
+int gen_pad_for(int box_rows, int G) { return (G + box_rows - 1) / box_rows * box_rows; }
 
 
 struct AttnPlan {
@@ -863,6 +868,7 @@ int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, 
     return st;
   }
   args.box_rows = box_rows_for(SPARSE, args.L, args.bs, args.g1 - args.g0);
+  args.gen_pad = gen_pad_for(args.box_rows, args.g1 - args.g0);
   CUtensorMap mk, mv;
   int st = make_kv_map(&mk, args.K, args.B * args.Hkv, args.L, D, args.box_rows);
   if (st != FOCUS_OK) return st;
@@ -951,8 +957,8 @@ extern "C" size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, in
                                                int P, int g0, int g1) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || acap <= 0 || Hq % Hkv || bs <= 0 || C <= 0 || S < 0) return 0;
   const int nb = (P + bs - 1) / bs;
-  const long kv_cap = static_cast<long>(std::min(C, std::max(nb, 0))) * ((bs + 7) & ~7) + ((g1 - g0 + 7) & ~7) +
-                      std::min(S, kMaxSinks);
+  const long kv_cap = static_cast<long>(std::min(C, std::max(nb, 0))) * ((bs + 7) & ~7) +
+                      gen_pad_for(box_rows_for(true, L, bs, g1 - g0), g1 - g0) + std::min(S, kMaxSinks);
   return plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(std::min<long>(kv_cap, 1 << 30)), false, L, S, C)
       .total;
 }
@@ -981,7 +987,8 @@ extern "C" int focus_sparse_attention(const focus_bf16* Q_active, const int32_t*
   }
   if (B == 0) return FOCUS_OK;
   const int nb = (P + bs - 1) / bs;
-  const long kv_cap = static_cast<long>(std::min(C, nb)) * ((bs + 7) & ~7) + ((g1 - g0 + 7) & ~7) + S;
+  const long kv_cap = static_cast<long>(std::min(C, nb)) * ((bs + 7) & ~7) +
+                      gen_pad_for(box_rows_for(true, L, bs, g1 - g0), g1 - g0) + S;
   FOCUS_CHECK_ARG(kv_cap < (1L << 30), "key set too large");
   const AttnPlan plan = plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(kv_cap), false, L, S, C);
   FOCUS_CHECK_ARG(ws_bytes >= plan.total && (plan.total == 0 || ws), "workspace too small: need %zu bytes, got %zu",

@@ -54,6 +54,7 @@ struct DecArgs {
   const int32_t* blocks;       // [B, Hkv, C]
   int B, Hq, Hkv, L, qcap, g;
   int box_rows;                // rows per TMA box (divides 128)
+  int gen_pad;                 // slots of the current block (multiple of box_rows)
   int S, C, bs, P, g0, g1;
   float scale_log2;
   int* dev_err;
@@ -121,49 +122,117 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int G = a.g1 - a.g0;
 
   // ---------------------------------------------------------------- prologue
+  // The producer warp initialises the barriers, builds the slot layout and issues the first
+  // STAGES tiles before the CTA barrier; meanwhile the MMA warp allocates tensor memory and
+  // the other warps stage Q.
+  volatile int* abort_flag = &bk->abort_flag;
+  const int BR = a.box_rows;
+  const int ngroups = 128 / BR;
+  const __nv_bfloat16* Kbh = a.K + static_cast<size_t>(bh) * a.L * D;
+  const __nv_bfloat16* Vbh = a.V + static_cast<size_t>(bh) * a.L * D;
+  int issued = 0;
+  SlotLayout sl_p{};
+  int p_begin = 0, p_n = 0;
+  // fetch tile `it` (ring stage it % STAGES) of this CTA's range: TMA boxes from parallel lanes
+  auto produce = [&](int it) {
+    const int s = it % STAGES;
+    const int slot0 = (p_begin + it) * 128;
+    uint8_t* dK = sK + s * SM::kTile;
+    uint8_t* dV = sV + s * SM::kTile;
+    const unsigned all_groups = (1u << ngroups) - 1u;     // ngroups <= 16
+    const int key0 = (lane < ngroups) ? group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + lane * BR) : -1;
+    const unsigned tma_mask = __ballot_sync(0xffffffffu, key0 >= 0) & all_groups;
+    if (lane == 0) mbar_expect_tx(&bk->full[s], __popc(tma_mask) * 2u * 2u * static_cast<uint32_t>(BR) * 128u);
+    __syncwarp();
+    // op j: group j / 4, atom (j / 2) & 1, K for even j, V for odd j; one op per lane
+    for (int j = lane; j < ngroups * 4; j += 32) {
+      const int grp = j >> 2;
+      if (!((tma_mask >> grp) & 1u)) continue;
+      const int k0 = group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + grp * BR);
+      const int at = (j >> 1) & 1;
+      const uint32_t off = at * (128 * 128) + grp * BR * 128;
+      if (j & 1) tma_load_3d(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, k0, bh);
+      else tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh);
+    }
+    if (SPARSE && tma_mask != all_groups) {
+      // sink rows (and rows past the end, zero-filled) by cp.async, 16 bytes per lane
+      for (int grp = 0; grp < ngroups; ++grp) {
+        if ((tma_mask >> grp) & 1u) continue;
+        for (int idx = lane; idx < BR * CH; idx += 32) {
+          const int rr = idx / CH, c = idx % CH;
+          const int row = grp * BR + rr;
+          const int key = sink_slot_key(sl_p, bk->sinks, slot0 + row);
+          const uint32_t src_bytes = key >= 0 ? 16u : 0u;
+          const size_t koff = static_cast<size_t>(key >= 0 ? key : 0) * D + c * 8;
+          cp_async16(smem_u32(dK + sw128_offset(row, c, 128)), Kbh + koff, src_bytes);
+          cp_async16(smem_u32(dV + sw128_offset(row, c, 128)), Vbh + koff, src_bytes);
+        }
+      }
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bk->full[s]);
+    __syncwarp();
+    ++issued;
+  };
+  if (warp == kDecProducerWarp) {
+    if (lane == 0) {
+      for (int st = 0; st < STAGES; ++st) {
+        mbar_init(&bk->full[st], 1);
+        mbar_init(&bk->empty[st], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bk->s_full[i], 1);
+        mbar_init(&bk->s_free[i], 4);
+        mbar_init(&bk->p_full[i], 4);
+        mbar_init(&bk->pv_done[i], 1);
+      }
+      mbar_init(&bk->drain, 1);
+      bk->abort_flag = 0;
+      fence_mbar_init();
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+    if (SPARSE) {
+      sl_p = build_sparse_layout(a.blocks + static_cast<size_t>(bh) * a.C, a.C,
+                                 a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs,
+                                 a.g0, a.g1, a.gen_pad, bk->blk, kDecMaxBlocks, bk->sinks, kDecMaxSinks, &bk->sl);
+    } else {
+      sl_p.n_slots = a.L;
+      if (lane == 0) bk->sl = sl_p;
+    }
+    const int tt = (sl_p.n_slots + 127) / 128;
+    const int tp = (tt + cs - 1) / cs;
+    p_begin = min(tt, rank * tp);
+    p_n = max(0, min(tt, p_begin + tp) - p_begin);
+    __syncwarp();
+    for (int it = 0; it < min(STAGES, p_n); ++it) produce(it);
+  }
   if (warp == kDecMmaWarp) {
     tmem_alloc(&bk->tmem_base, SM::kTmemCols);
     tmem_relinquish();
   }
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&bk->full[s], 1);
-      mbar_init(&bk->empty[s], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bk->s_full[i], 1);
-      mbar_init(&bk->s_free[i], 4);
-      mbar_init(&bk->p_full[i], 4);
-      mbar_init(&bk->pv_done[i], 1);
-    }
-    mbar_init(&bk->drain, 1);
-    bk->abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (SPARSE) {
-    if (warp == 0)
-      build_sparse_layout(a.blocks + static_cast<size_t>(bh) * a.C, a.C,
-                          a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs, a.g0,
-                          a.g1, bk->blk, kDecMaxBlocks, bk->sinks, kDecMaxSinks, &bk->sl);
-  } else if (threadIdx.x == 0) {
-    bk->sl.n_slots = a.L;
-  }
-  // Q rows (query q <-> head kvh*g + q/qcap, position q%qcap) as a K-major SW128 B operand
-  for (int idx = threadIdx.x; idx < NQ * CH; idx += kDecThreads) {
-    const int q = idx / CH, c = idx % CH;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (q < n_rows) {
-      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
-      if (i < nq_b)
+  if (warp != kDecProducerWarp) {
+    // Q rows (query q <-> head kvh*g + q/qcap, position q%qcap) as a K-major SW128 B
+    // operand; rows are loaded before the valid count is known and masked afterwards
+    const int qt = warp < kDecProducerWarp ? threadIdx.x : threadIdx.x - 32;   // 0..159 without the producer
+    for (int idx = qt; idx < NQ * CH; idx += kDecThreads - 32) {
+      const int q = idx / CH, c = idx % CH;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (q < n_rows) {
+        const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
         v = __ldg(reinterpret_cast<const uint4*>(a.Q + ((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D) + c);
+        if (i >= nq_b) v = make_uint4(0u, 0u, 0u, 0u);
+      }
+      *reinterpret_cast<uint4*>(sQ + sw128_offset(q, c, NQ)) = v;
     }
-    *reinterpret_cast<uint4*>(sQ + sw128_offset(q, c, NQ)) = v;
+    if (threadIdx.x < NQ) {
+      bk->mref[threadIdx.x] = -INFINITY;
+      bk->alpha[threadIdx.x] = 1.f;
+    }
+    fence_proxy_async_smem();
   }
-  if (threadIdx.x < NQ) {
-    bk->mref[threadIdx.x] = -INFINITY;
-    bk->alpha[threadIdx.x] = 1.f;
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -174,73 +243,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int tps = (total_tiles + cs - 1) / cs;
   const int t_begin = min(total_tiles, rank * tps);
   const int n_it = max(0, min(total_tiles, t_begin + tps) - t_begin);
-  volatile int* abort_flag = &bk->abort_flag;
   float lsum[NQ];
 #pragma unroll
   for (int q = 0; q < NQ; ++q) lsum[q] = 0.f;
 
   if (warp == kDecProducerWarp) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-    }
-    const int BR = a.box_rows;
-    const int ngroups = 128 / BR;
-    const __nv_bfloat16* Kbh = a.K + static_cast<size_t>(bh) * a.L * D;
-    const __nv_bfloat16* Vbh = a.V + static_cast<size_t>(bh) * a.L * D;
-    int issued = 0;
-    for (int it = 0; it < n_it; ++it) {
+    for (int it = STAGES; it < n_it; ++it) {
       const int s = it % STAGES;
-      if (it >= STAGES &&
-          !__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
+      if (!__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
                                              DEV_ERR_TIMEOUT_PRODUCER)))
         break;
-      const int slot0 = (t_begin + it) * 128;
-      uint8_t* dK = sK + s * SM::kTile;
-      uint8_t* dV = sV + s * SM::kTile;
-      // TMA for contiguous runs
-      if (lane == 0) {
-        uint32_t tma_groups = 0;
-        for (int grp = 0; grp < ngroups; ++grp)
-          if (group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR) >= 0) ++tma_groups;
-        mbar_expect_tx(&bk->full[s], tma_groups * 2u * 2u * static_cast<uint32_t>(BR) * 128u);
-        for (int grp = 0; grp < ngroups; ++grp) {
-          const int key0 = group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR);
-          if (key0 < 0) continue;
-#pragma unroll
-          for (int at = 0; at < 2; ++at) {
-            const uint32_t off = at * (128 * 128) + grp * BR * 128;
-            tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, key0, bh);
-            tma_load_3d(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, key0, bh);
-          }
-        }
-      }
-      if (SPARSE) {
-        // sink rows (and rows past the end, zero-filled) by cp.async, 16 bytes per lane
-        bool any_rows = false;
-        for (int grp = 0; grp < ngroups; ++grp) {
-          if (group_key0<SPARSE>(sl, bk->blk, a.bs, a.g0, slot0 + grp * BR) >= 0) continue;
-          any_rows = true;
-          for (int idx = lane; idx < BR * CH; idx += 32) {
-            const int rr = idx / CH, c = idx % CH;
-            const int row = grp * BR + rr;
-            const int key = sink_slot_key(sl, bk->sinks, slot0 + row);
-            const uint32_t src_bytes = key >= 0 ? 16u : 0u;
-            const size_t koff = static_cast<size_t>(key >= 0 ? key : 0) * D + c * 8;
-            cp_async16(smem_u32(dK + sw128_offset(row, c, 128)), Kbh + koff, src_bytes);
-            cp_async16(smem_u32(dV + sw128_offset(row, c, 128)), Vbh + koff, src_bytes);
-          }
-        }
-        if (any_rows) {
-          cp_async_wait_all();
-          fence_proxy_async_smem();
-        }
-        __syncwarp();
-      }
-      if (lane == 0) mbar_arrive(&bk->full[s]);
-      __syncwarp();
-      ++issued;
+      produce(it);
     }
     if (lane == 0)
       for (int j = max(0, issued - STAGES); j < issued; ++j) dec_wait_drain(&bk->full[j % STAGES], (j / STAGES) & 1);
@@ -433,7 +447,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   tc_fence_after();
   const bool have_o = (n_it > 0) && !bk->abort_flag;
   // index (q / cs) * cs + src < NQ + cs <= NQ + 8: (NQ + 8) x D floats fit in the V ring
-  static_assert((NQ + 8) * (D + 2) * 4 <= STAGES * SM::kTile, "receive buffer exceeds the V ring");
+  static_assert((NQ + 8) * (D + 2) * 4 + NQ * 8 * 4 <= STAGES * SM::kTile, "receive buffer exceeds the V ring");
   float* recv_o = reinterpret_cast<float*>(sV);    // [(q / cs) * cs + src][D]
   float* recv_ml = recv_o + (NQ + 8) * D;          // [(q / cs) * cs + src][2]
   float ov[NQ];
@@ -483,34 +497,44 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
   if (cs > 1) cluster_sync();        // pushes visible to their owners
   else __syncthreads();
+  // per-query merge weights, one thread per owned query: w[src] = 2^(m_src - M) / l
+  float* mw = recv_ml + (NQ + 8) * 2;            // [owned query][8] weights
   if (warp < 4) {
     const int t = threadIdx.x;
-    for (int q = rank; q < n_rows; q += cs) {
+    const int q = rank + t * cs;
+    if (q < n_rows) {
       const int slot = q / cs;
-      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
-      const size_t row = (static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i;
-      float o = 0.f, lse = -INFINITY;
-      if (i < nq_b) {
-        float M = -INFINITY;
-        for (int r = 0; r < cs; ++r) {
+      float M = -INFINITY;
+      for (int r = 0; r < cs; ++r)
+        if (recv_ml[(slot * cs + r) * 2 + 1] > 0.f) M = fmaxf(M, recv_ml[(slot * cs + r) * 2]);
+      float l = 0.f;
+      float w[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        w[r] = 0.f;
+        if (r < cs && M > -INFINITY) {
           const float lr = recv_ml[(slot * cs + r) * 2 + 1];
-          if (lr > 0.f) M = fmaxf(M, recv_ml[(slot * cs + r) * 2]);
-        }
-        if (M > -INFINITY) {
-          float l = 0.f;
-          for (int r = 0; r < cs; ++r) {
-            const float lr = recv_ml[(slot * cs + r) * 2 + 1];
-            if (!(lr > 0.f)) continue;
-            const float w = exp2_approx(recv_ml[(slot * cs + r) * 2] - M);
-            l += w * lr;
-            o += w * recv_o[(slot * cs + r) * D + t];
+          if (lr > 0.f) {
+            w[r] = exp2_approx(recv_ml[(slot * cs + r) * 2] - M);
+            l += w[r] * lr;
           }
-          o /= l;
-          lse = M + __log2f(l);
         }
       }
-      a.O[row * D + t] = __float2bfloat16_rn(o);
-      if (t == 0 && a.lse_out && i < nq_b) a.lse_out[row] = lse;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r < cs) mw[t * 8 + r] = w[r] * inv;
+      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
+      if (a.lse_out && i < nq_b) a.lse_out[(static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i] = M + __log2f(l);
+    }
+    named_bar_sync(1, 128);
+    for (int qi = 0, q = rank; q < n_rows; ++qi, q += cs) {
+      const int slot = q / cs;
+      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
+      float o = 0.f;
+      if (i < nq_b)
+        for (int r = 0; r < cs; ++r) o += mw[qi * 8 + r] * recv_o[(slot * cs + r) * D + t];
+      a.O[((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D + t] = __float2bfloat16_rn(o);
     }
   }
   tc_fence_before();
@@ -666,10 +690,12 @@ int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bflo
   int cap = 128;
   while (cap > L) cap >>= 1;
   if (sparse) {
-    const int pad_bs = (bs + 7) & ~7, pad_g = (g1 - g0 + 7) & ~7;
-    a.box_rows = std::min(pow2_divisor(pad_bs, cap), pow2_divisor(pad_g, cap));
+    // boxes stay inside one kept block; the current block is padded to whole boxes
+    a.box_rows = pow2_divisor((bs + 7) & ~7, cap);
+    a.gen_pad = (g1 - g0 + a.box_rows - 1) / a.box_rows * a.box_rows;
   } else {
     a.box_rows = cap;
+    a.gen_pad = 0;
   }
   const int nrows = a.g * qcap;
   if (nrows <= 32)

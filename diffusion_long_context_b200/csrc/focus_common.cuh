@@ -14,7 +14,7 @@
 
 #include <utility>
 
-#include "../../include/focus.h"
+#include "focus.h"
 
 namespace focus {
 

@@ -4,7 +4,7 @@
 // Sparse (Focus-dLLM method steps (5): I_p = sinks U kept prompt blocks U current
 // block, each key once): slots are laid out as
 //   [ kept block 0 | kept block 1 | ... ]  each padded to pad_bs = round_up(bs, 8)
-//   [ current block [g0, g1) ]             padded to round_up(G, 8)
+//   [ current block [g0, g1) ]             padded to gen_pad slots (a multiple of 8 >= G)
 //   [ de-duplicated sinks ]                sinks inside a kept block or the current
 //                                          block, out-of-range and repeated entries dropped
 // Padding slots are invalid (masked out of the softmax). Every box_rows-aligned group of
@@ -29,10 +29,12 @@ struct SlotLayout {
 // One warp builds the layout of (b, h): copies the kept-block list to s_blk (up to
 // max_blocks entries) and the de-duplicated sinks to s_sinks (up to max_sinks). The block
 // list has its valid entries first, ascending, then -1; sinks are ascending among valid
-// entries. Lane 0 writes *out.
-__device__ __forceinline__ void build_sparse_layout(const int32_t* blk_g, int C, const int32_t* snk_g, int S, int L,
-                                                    int P, int bs, int g0, int g1, int* s_blk, int max_blocks,
-                                                    int* s_sinks, int max_sinks, SlotLayout* out) {
+// entries. gen_pad = slots given to the current block. Lane 0 writes *out; the layout is
+// also returned to every lane of the warp.
+__device__ __forceinline__ SlotLayout build_sparse_layout(const int32_t* blk_g, int C, const int32_t* snk_g, int S,
+                                                          int L, int P, int bs, int g0, int g1, int gen_pad, int* s_blk,
+                                                          int max_blocks, int* s_sinks, int max_sinks,
+                                                          SlotLayout* out) {
   const int lane = threadIdx.x & 31;
   int nvb = 0;
   for (int i0 = 0; i0 < C; i0 += 32) {
@@ -74,17 +76,16 @@ __device__ __forceinline__ void build_sparse_layout(const int32_t* blk_g, int C,
     nf += __popc(m);
     prev_last = __shfl_sync(0xffffffffu, j, 31);
   }
-  if (lane == 0) {
-    const int pad_bs = (bs + 7) & ~7;
-    const int G = g1 - g0;
-    out->pad_bs = pad_bs;
-    out->nvb = nvb;
-    out->last_size = last_size;
-    out->gen_start = nvb * pad_bs;
-    out->sink_start = out->gen_start + ((G + 7) & ~7);
-    out->n_fsinks = min(nf, max_sinks);
-    out->n_slots = out->sink_start + out->n_fsinks;
-  }
+  SlotLayout sl;
+  sl.pad_bs = (bs + 7) & ~7;
+  sl.nvb = nvb;
+  sl.last_size = last_size;
+  sl.gen_start = nvb * sl.pad_bs;
+  sl.sink_start = sl.gen_start + gen_pad;
+  sl.n_fsinks = min(nf, max_sinks);
+  sl.n_slots = sl.sink_start + sl.n_fsinks;
+  if (lane == 0) *out = sl;
+  return sl;
 }
 
 // First key of the contiguous run starting at group slot gs (box-aligned), or -1 when the
