@@ -331,6 +331,7 @@ def run_ours(args):
         "select_and_gather": graph_ms([step.select], reps),
         "dense_attention": graph_ms([lambda l=l: step.dense_layer(l) for l in range(c.l_dense)], reps),
         "dense_attention_colsum_sinks": graph_ms([lambda: step.dense_layer(c.l_dense)], reps),
+        "sparse_layer_fused": graph_ms([lambda l=l: step.sparse_layer_fused(l) for l in step.sparse_layers], reps),
         "block_select": graph_ms([lambda l=l: step.block_select_layer(l) for l in step.sparse_layers], reps),
         "sparse_attention": graph_ms([lambda l=l: step.sparse_attention_layer(l) for l in step.sparse_layers], reps),
     }
@@ -344,10 +345,12 @@ def run_ours(args):
     sparse_bytes = mean_ip * c.d * 2 * 2 + 2 * c.B * c.Hq * A * c.d * 2
     sparse_flops = 4.0 * A * g * mean_ip * c.d
     dense_bytes = c.B * c.Hkv * c.L * c.d * 2 * 2 + 2 * c.B * c.Hq * A * c.d * 2
+    kbar_bytes = c.B * c.Hkv * c.nb * c.d * 4
+    # the step runs focus_block_select then focus_sparse_attention per sparse layer; the
+    # roofline reports the attention launch (gathered K/V + Q + O bytes)
     t_sp = call_ms["sparse_attention"] * 1e-3
     achieved = sparse_bytes / t_sp / 1e9
     # step roofline: slower of bytes at HBM peak and flops at the tensor peak, summed over calls
-    kbar_bytes = c.B * c.Hkv * c.nb * c.d * 4
     n_dense, n_sparse = c.l_dense + 1, c.n_layers - c.l_dense - 1
     colsum_bytes = c.B * c.Hkv * c.L * c.d * 2
     step_bytes = n_dense * dense_bytes + colsum_bytes + n_sparse * (sparse_bytes + kbar_bytes)
@@ -427,7 +430,8 @@ def run_ours(args):
                        "replay": "one CUDA graph per step", "parallelism": f"replicas x{ws}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": None,
-                         "kernel": "focus_sparse_attention, one layer (CUDA-graph replay of all sparse layers)",
+                         "kernel": "focus_sparse_attention (decode kernel, cluster split), one layer; CUDA-graph "
+                                   "replay of all sparse layers",
                          "bytes_per_launch": sparse_bytes, "flops_per_launch": sparse_flops,
                          "launch_ms": call_ms["sparse_attention"], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "roofline_ms": step_roof_ms, "frac": step_roof_ms / ms_step},

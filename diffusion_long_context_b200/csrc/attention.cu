@@ -37,7 +37,8 @@ bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C);
 int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                      __nv_bfloat16* O, float* lse_out, const int32_t* sinks, const int32_t* blocks, int S, int C, int bs,
                      int P, int g0, int g1, bool sparse, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
-                     cudaStream_t stream);
+                     cudaStream_t stream, const float* kbar = nullptr, int nb = 0, int32_t* blocks_out = nullptr);
+bool decode_fused_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C, int nb);
 
 constexpr int kBM = 128;            // query rows per CTA (tcgen05 M)
 constexpr int kBN = 128;            // keys per tile
@@ -1018,4 +1019,31 @@ extern "C" int focus_sparse_attention(const focus_bf16* Q_active, const int32_t*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? run_attention<128, true>(a, plan, ws, nullptr, s)
                   : run_attention<64, true>(a, plan, ws, nullptr, s);
+}
+
+extern "C" int focus_sparse_attention_fused(const focus_bf16* Q_active, const int32_t* n_active, const focus_bf16* K,
+                                            const focus_bf16* V, const float* kbar, int nb, int C,
+                                            const int32_t* sinks, int S, int bs, int P, int g0, int g1, int B, int Hq,
+                                            int Hkv, int L, int d, int acap, float scale, int32_t* blocks,
+                                            focus_bf16* O_active, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_common(Q_active, K, V, O_active, B, Hq, Hkv, L, d, acap);
+  if (st != FOCUS_OK) return st;
+  FOCUS_CHECK_ARG(n_active && kbar && blocks && (S == 0 || sinks), "null pointer argument");
+  FOCUS_CHECK_ARG(aligned16(kbar), "kbar must be 16-byte aligned");
+  FOCUS_CHECK_ARG(nb == (P + bs - 1) / bs && nb >= 1, "nb (%d) must equal ceil(P / bs)", nb);
+  if (!decode_fused_supported(d, Hq, Hkv, acap, L, S, C, nb)) {
+    // shapes the fused kernel does not take: the two calls in sequence
+    st = focus_block_select(Q_active, n_active, kbar, B, Hq, Hkv, d, acap, nb, C, blocks, nullptr, stream);
+    if (st != FOCUS_OK) return st;
+    return focus_sparse_attention(Q_active, n_active, K, V, sinks, S, blocks, C, bs, P, g0, g1, B, Hq, Hkv, L, d,
+                                  acap, scale, O_active, ws, ws_bytes, stream);
+  }
+  FOCUS_CHECK_ARG(bs >= 1 && C >= 1 && S >= 0, "bad bs=%d C=%d S=%d", bs, C, S);
+  FOCUS_CHECK_ARG(0 <= P && P <= g0 && g0 < g1 && g1 <= L, "need 0 <= P <= g0 < g1 <= L (P=%d g0=%d g1=%d L=%d)", P,
+                  g0, g1, L);
+  if (B == 0) return FOCUS_OK;
+  return decode_attention(reinterpret_cast<const __nv_bfloat16*>(Q_active), n_active,
+                          reinterpret_cast<const __nv_bfloat16*>(K), reinterpret_cast<const __nv_bfloat16*>(V),
+                          reinterpret_cast<__nv_bfloat16*>(O_active), nullptr, sinks, nullptr, S, C, bs, P, g0, g1, true,
+                          B, Hq, Hkv, L, acap, scale * kLog2e, static_cast<cudaStream_t>(stream), kbar, nb, blocks);
 }

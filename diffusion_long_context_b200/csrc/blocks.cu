@@ -52,7 +52,9 @@ __global__ void __launch_bounds__(256) block_means_kernel(const __nv_bfloat16* _
 
 constexpr int kSelectThreads = 512;
 
-// One CTA per (sequence, KV head): qbar, R over all blocks, top-C.
+// One cluster of `gridDim.x` CTAs per (sequence, KV head). Every CTA forms qbar and scores
+// its share of the blocks (8 kbar rows in flight per warp), pushing R into CTA 0's shared
+// memory through DSMEM; after a cluster barrier CTA 0 selects the top-C.
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
     const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ n_active, const float* __restrict__ kbar, int Hq,
@@ -60,28 +62,39 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   griddep_wait();               // inputs may come from the previous kernel on the stream
   griddep_launch_dependents();
   constexpr int PARTS = kSelectThreads / D;
-  extern __shared__ float s_R[];           // [nb]
+  extern __shared__ float s_R[];           // [nb], gathered in CTA 0
   __shared__ float s_part[PARTS][D];
   __shared__ float s_qbar[D];
   __shared__ TopkShared tk;
-  const int bh = blockIdx.x;
+  const int cs = gridDim.x, rank = blockIdx.x;
+  const int bh = blockIdx.y;
   const int b = bh / Hkv, h = bh % Hkv;
   const int g = Hq / Hkv;
-  const int A = n_active[b];
+  const int A = min(n_active[b], acap);
   const int dim = threadIdx.x % D, part = threadIdx.x / D;
   float acc = 0.f;
   const int rows = g * A;
-  for (int r = part; r < rows; r += PARTS) {
-    const int hq = h * g + r / A, i = r % A;
-    acc += __bfloat162float(Q[((static_cast<size_t>(b) * Hq + hq) * acap + i) * D + dim]);
+  for (int r0 = part; r0 < rows; r0 += PARTS * 8) {       // 8 rows in flight per thread
+    __nv_bfloat16 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int r = r0 + PARTS * u;
+      v[u] = __float2bfloat16_rn(0.f);
+      if (r < rows) {
+        const int hq = h * g + r / A, i = r % A;
+        v[u] = Q[((static_cast<size_t>(b) * Hq + hq) * acap + i) * D + dim];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += __bfloat162float(v[u]);
   }
   s_part[part][dim] = acc;
   __syncthreads();
   if (threadIdx.x < D) {
-    float s = 0.f;
+    float sum = 0.f;
 #pragma unroll
-    for (int p = 0; p < PARTS; ++p) s += s_part[p][threadIdx.x];
-    s_qbar[threadIdx.x] = rows > 0 ? s / static_cast<float>(rows) : 0.f;
+    for (int p = 0; p < PARTS; ++p) sum += s_part[p][threadIdx.x];
+    s_qbar[threadIdx.x] = rows > 0 ? sum / static_cast<float>(rows) : 0.f;
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,16 +103,19 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   float4 qv = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane < LANES) qv = reinterpret_cast<const float4*>(s_qbar)[lane];
   const float* kb = kbar + static_cast<size_t>(bh) * nb * D;
-  // 8 rows of kbar in flight per warp: 16 warps cover 128 blocks per pass
+  const int chunk = (nb + cs - 1) / cs;
+  const int j_begin = rank * chunk, j_end = min(nb, j_begin + chunk);
+  const uint32_t sR0 = smem_u32(s_R);
   constexpr int UNR = 8;
   constexpr int NW = kSelectThreads / 32;
-  for (int j0 = warp * UNR; j0 < nb; j0 += NW * UNR) {
+  for (int j0 = j_begin + warp * UNR; j0 < j_end; j0 += NW * UNR) {
     float4 kv[UNR];
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
       const int j = j0 + u;
-      kv[u] = (j < nb && lane < LANES) ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D) + lane)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      kv[u] = (j < j_end && lane < LANES)
+                  ? __ldg(reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D) + lane)
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < UNR; ++u) {
@@ -107,14 +123,20 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
       const int j = j0 + u;
-      if (lane == 0 && j < nb) {
+      if (lane == 0 && j < j_end) {
         const float R = p * inv_sqrt_d;
-        s_R[j] = R;
+        if (cs > 1) {
+          asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_addr(sR0 + 4u * j, 0)), "f"(R) : "memory");
+        } else {
+          s_R[j] = R;
+        }
         if (scores) scores[static_cast<size_t>(bh) * nb + j] = R;
       }
     }
   }
-  __syncthreads();
+  if (cs > 1) cluster_sync();   // every share of R is in CTA 0
+  else __syncthreads();
+  if (rank != 0) return;
   block_topk_ascending([&](int i) { return float_order_key(s_R[i]); }, nb, C, blocks + static_cast<size_t>(bh) * C, C,
                        tk);
 }
@@ -155,6 +177,7 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
   FOCUS_CHECK_ARG(B >= 0 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && acap >= 1 && nb >= 1 && C >= 1,
                   "bad sizes (Hq=%d Hkv=%d acap=%d nb=%d C=%d)", Hq, Hkv, acap, nb, C);
   FOCUS_CHECK_ARG(aligned16(kbar), "kbar must be 16-byte aligned");
+  FOCUS_CHECK_ARG(static_cast<long long>(B) * Hkv < 65536, "B*Hkv must be < 65536");
   if (d != 64 && d != 128) {
     set_error("head dim %d unsupported (64 or 128)", d);
     return FOCUS_ERR_UNSUPPORTED;
@@ -167,6 +190,10 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
   const size_t smem = static_cast<size_t>(nb) * sizeof(float);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(Q_active);
+  // cluster of cs CTAs per (sequence, KV head), cs a power of two with B*Hkv*cs <= SMs
+  const int units = B * Hkv;
+  int cs = 1;
+  while (cs < 8 && units * cs * 2 <= device_sm_count() && (nb + cs * 2 - 1) / (cs * 2) >= 16) cs *= 2;
   cudaError_t err;
   if (d == 128) {
     static bool cfg = false;
@@ -174,16 +201,16 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
       cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
       cfg = true;
     }
-    err = launch_k(block_select_kernel<128>, dim3(B * Hkv), dim3(kSelectThreads), smem, s, q, n_active, kbar, Hq,
-                   Hkv, acap, nb, C, blocks, scores_opt);
+    err = launch_k_cluster(block_select_kernel<128>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
+                           n_active, kbar, Hq, Hkv, acap, nb, C, blocks, scores_opt);
   } else {
     static bool cfg = false;
     if (!cfg) {
       cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
       cfg = true;
     }
-    err = launch_k(block_select_kernel<64>, dim3(B * Hkv), dim3(kSelectThreads), smem, s, q, n_active, kbar, Hq,
-                   Hkv, acap, nb, C, blocks, scores_opt);
+    err = launch_k_cluster(block_select_kernel<64>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
+                           n_active, kbar, Hq, Hkv, acap, nb, C, blocks, scores_opt);
   }
   note_launch();
   if (err != cudaSuccess) {

@@ -33,6 +33,7 @@
 
 #include "focus_common.cuh"
 #include "slots.cuh"
+#include "topk.cuh"
 
 namespace focus {
 
@@ -51,7 +52,10 @@ struct DecArgs {
   __nv_bfloat16* O;            // [B, Hq, qcap, D]
   float* lse_out;              // [B, Hq, qcap] log2 domain, or null
   const int32_t* sinks;        // [B, Hkv, S]
-  const int32_t* blocks;       // [B, Hkv, C]
+  const int32_t* blocks;       // [B, Hkv, C] (unfused sparse)
+  const float* kbar;           // [B, Hkv, nb, D] (fused sparse: relevance + top-C in the prologue)
+  int32_t* blocks_out;         // [B, Hkv, C] kept blocks written by the fused kernel, or null
+  int nb;
   int B, Hq, Hkv, L, qcap, g;
   int box_rows;                // rows per TMA box (divides 128)
   int gen_pad;                 // slots of the current block (multiple of box_rows)
@@ -73,6 +77,9 @@ struct __align__(8) DecBook {
   float red[4][64];
   int blk[kDecMaxBlocks];
   int sinks[kDecMaxSinks];
+  TopkShared tk;
+  uint32_t tile_ctr;       // next dynamically claimed tile (CTA 0 of the cluster)
+  int stage_tile[4];       // tile held by each ring stage, -1 = no more tiles
 };
 
 template <int NQ, int STAGES>
@@ -85,6 +92,8 @@ struct DecSmem {
   static constexpr uint32_t kBook = kP + 2 * NQ * 256;
   static constexpr uint32_t kBytes = kBook + sizeof(DecBook) + 1024;
   static constexpr uint32_t kTmemCols = (3 * NQ <= 128) ? 128 : 256;
+  static_assert(kBytes <= 232448, "decode kernel exceeds the 227 KB of shared memory per CTA");
+  static_assert(2 * NQ * 256 >= 4 * 4096, "fused relevance scores must fit in the P buffers");
 };
 
 __device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
@@ -95,7 +104,9 @@ __device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
-template <int NQ, int STAGES, bool SPARSE>
+constexpr int kDecMaxNb = 4096;   // fused relevance scores held in the P buffers
+
+template <int NQ, int STAGES, bool SPARSE, bool FUSED>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const DecArgs a) {
@@ -132,11 +143,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const __nv_bfloat16* Vbh = a.V + static_cast<size_t>(bh) * a.L * D;
   int issued = 0;
   SlotLayout sl_p{};
-  int p_begin = 0, p_n = 0;
-  // fetch tile `it` (ring stage it % STAGES) of this CTA's range: TMA boxes from parallel lanes
-  auto produce = [&](int it) {
+  int p_n = 0;                 // tiles of this (b, h)
+  bool p_more = true;          // the end marker is not issued yet
+  // fetch tile `tile` into ring stage `it % STAGES`: TMA boxes from parallel lanes
+  auto produce = [&](int it, int tile) {
     const int s = it % STAGES;
-    const int slot0 = (p_begin + it) * 128;
+    const int slot0 = tile * 128;
     uint8_t* dK = sK + s * SM::kTile;
     uint8_t* dV = sV + s * SM::kTile;
     const unsigned all_groups = (1u << ngroups) - 1u;     // ngroups <= 16
@@ -172,10 +184,110 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       fence_proxy_async_smem();
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bk->full[s]);
+    if (lane == 0) {
+      bk->stage_tile[s] = tile;
+      mbar_arrive(&bk->full[s]);
+    }
     __syncwarp();
     ++issued;
   };
+  // no more tiles: stage `it % STAGES` carries the end marker (plain arrive, no bytes)
+  auto produce_end = [&](int it) {
+    if (lane == 0) {
+      bk->stage_tile[it % STAGES] = -1;
+      mbar_arrive(&bk->full[it % STAGES]);
+    }
+    __syncwarp();
+  };
+  // Tiles of this (b, h): CTA `rank` takes tiles rank, rank + cs, ... for its first STAGES
+  // stages; after that every CTA claims the next tile from the counter in CTA 0.
+  // The counter's initialisation is ordered before any claim by a cluster barrier: the
+  // relevance prologue's own, else a split barrier around the prologue.
+  if (threadIdx.x == 0 && rank == 0) bk->tile_ctr = static_cast<uint32_t>(cs * STAGES);
+  if (!FUSED && cs > 1) cluster_arrive();
+  if (FUSED) {
+    // ---- block relevance R_b = qbar . kbar_b / sqrt(d) and top-C (method steps (4)) ----
+    // qbar over the active rows of this KV group; partial sums in the (still idle) K ring
+    float* s_part = reinterpret_cast<float*>(sK);            // [3][D]
+    float* s_qbar = s_part + 3 * D;                            // [D]
+    float* s_R = reinterpret_cast<float*>(sP);                 // [nb], every CTA holds all of R
+    const int rows = a.g * nq_b;
+    const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
+    const float* kb = a.kbar + static_cast<size_t>(bh) * a.nb * D;
+    const int chunk = (a.nb + cs - 1) / cs;
+    const int j_begin = rank * chunk, j_end = min(a.nb, j_begin + chunk);
+    uint32_t* s_key = reinterpret_cast<uint32_t*>(s_R);
+    const uint32_t sK0 = smem_u32(s_key);
+    // this thread's first kbar row is fetched before qbar is known (the two loads overlap)
+    int j = j_begin + threadIdx.x;
+    float4 kv[D / 4];
+    if (j < j_end) {
+      const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c) kv[c] = __ldg(row + c);
+    }
+    {
+      // qbar: 3 row groups x 64 dim pairs; 8 rows in flight per thread
+      const int t = threadIdx.x, dp = t % 64, rg = t / 64;
+      float2 acc = make_float2(0.f, 0.f);
+      for (int r0 = rg; r0 < rows; r0 += 3 * 8) {
+        __nv_bfloat162 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int r = r0 + 3 * u;
+          v[u] = __floats2bfloat162_rn(0.f, 0.f);
+          if (r < rows) {
+            const int hq = kvh * a.g + r / nq_b, i = r % nq_b;
+            v[u] = *reinterpret_cast<const __nv_bfloat162*>(
+                a.Q + ((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D + 2 * dp);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float2 f = __bfloat1622float2(v[u]);
+          acc.x += f.x;
+          acc.y += f.y;
+        }
+      }
+      s_part[rg * D + 2 * dp] = acc.x;
+      s_part[rg * D + 2 * dp + 1] = acc.y;
+    }
+    __syncthreads();
+    if (threadIdx.x < D) {
+      const float q = (s_part[threadIdx.x] + s_part[D + threadIdx.x]) + s_part[2 * D + threadIdx.x];
+      s_qbar[threadIdx.x] = rows > 0 ? q / static_cast<float>(rows) : 0.f;
+    }
+    __syncthreads();
+    // R of this CTA's share of the blocks, one kbar row per thread; the order key of every
+    // score is broadcast to each CTA of the cluster
+    while (j < j_end) {
+      float p = 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 4; ++c) {
+        const float4 qv = reinterpret_cast<const float4*>(s_qbar)[c];
+        p += qv.x * kv[c].x + qv.y * kv[c].y + qv.z * kv[c].z + qv.w * kv[c].w;
+      }
+      const uint32_t key = float_order_key(p * inv_sqrt_d);
+      if (cs > 1) {
+        for (int r = 0; r < cs; ++r)
+          asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dsmem_addr(sK0 + 4u * j, r)), "r"(key) : "memory");
+      } else {
+        s_key[j] = key;
+      }
+      j += kDecThreads;
+      if (j < j_end) {
+        const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
+#pragma unroll
+        for (int c = 0; c < D / 4; ++c) kv[c] = __ldg(row + c);
+      }
+    }
+    if (cs > 1) cluster_sync();   // every CTA holds all nb keys
+    else __syncthreads();
+    block_topk_ascending([&](int i) { return s_key[i]; }, a.nb, a.C, bk->blk, a.C, bk->tk);
+    __syncthreads();
+    if (rank == 0 && a.blocks_out)
+      for (int i = threadIdx.x; i < a.C; i += kDecThreads) a.blocks_out[static_cast<size_t>(bh) * a.C + i] = bk->blk[i];
+  }
   if (warp == kDecProducerWarp) {
     if (lane == 0) {
       for (int st = 0; st < STAGES; ++st) {
@@ -195,19 +307,24 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tma_prefetch_desc(&tmV);
     }
     if (SPARSE) {
-      sl_p = build_sparse_layout(a.blocks + static_cast<size_t>(bh) * a.C, a.C,
+      sl_p = build_sparse_layout(FUSED ? bk->blk : a.blocks + static_cast<size_t>(bh) * a.C, a.C,
                                  a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs,
                                  a.g0, a.g1, a.gen_pad, bk->blk, kDecMaxBlocks, bk->sinks, kDecMaxSinks, &bk->sl);
     } else {
       sl_p.n_slots = a.L;
       if (lane == 0) bk->sl = sl_p;
     }
-    const int tt = (sl_p.n_slots + 127) / 128;
-    const int tp = (tt + cs - 1) / cs;
-    p_begin = min(tt, rank * tp);
-    p_n = max(0, min(tt, p_begin + tp) - p_begin);
+    p_n = (sl_p.n_slots + 127) / 128;
     __syncwarp();
-    for (int it = 0; it < min(STAGES, p_n); ++it) produce(it);
+    for (int it = 0; it < STAGES; ++it) {
+      const int tile = rank + it * cs;
+      if (tile >= p_n) {
+        produce_end(it);
+        p_more = false;
+        break;
+      }
+      produce(it, tile);
+    }
   }
   if (warp == kDecMmaWarp) {
     tmem_alloc(&bk->tmem_base, SM::kTmemCols);
@@ -234,30 +351,48 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     fence_proxy_async_smem();
   }
   tc_fence_before();
+  if (!FUSED && cs > 1) cluster_wait();
   __syncthreads();
   tc_fence_after();
 
   const uint32_t tmem = bk->tmem_base;
   const SlotLayout sl = bk->sl;
-  const int total_tiles = (sl.n_slots + 127) / 128;
-  const int tps = (total_tiles + cs - 1) / cs;
-  const int t_begin = min(total_tiles, rank * tps);
-  const int n_it = max(0, min(total_tiles, t_begin + tps) - t_begin);
+  int n_it = 0;                                  // tiles this CTA processed (set by each role)
   float lsum[NQ];
 #pragma unroll
   for (int q = 0; q < NQ; ++q) lsum[q] = 0.f;
 
   if (warp == kDecProducerWarp) {
     // ------------------------------------------------------------ producer
-    for (int it = STAGES; it < n_it; ++it) {
-      const int s = it % STAGES;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
-                                             DEV_ERR_TIMEOUT_PRODUCER)))
-        break;
-      produce(it);
+    // A wait that ran out raises the abort flag, which ends the other roles' loops; the
+    // end marker is then not issued.
+    bool drained_marker = !p_more;
+    if (p_more) {
+      const uint32_t ctr = smem_u32(&bk->tile_ctr);
+      int next = 0;
+      if (lane == 0) next = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
+      next = __shfl_sync(0xffffffffu, next, 0);
+      for (int it = STAGES;; ++it) {
+        const int s = it % STAGES;
+        if (!__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
+                                               DEV_ERR_TIMEOUT_PRODUCER)))
+          break;
+        if (next >= p_n) {
+          produce_end(it);
+          drained_marker = true;
+          break;
+        }
+        const int tile = next;
+        if (lane == 0) next = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));   // claim ahead
+        next = __shfl_sync(0xffffffffu, next, 0);
+        produce(it, tile);
+      }
     }
+    // wait for the copies still in flight; the end marker (issue index `issued`) shares its
+    // stage with tile issued - STAGES, which had completed before the marker was issued
     if (lane == 0)
-      for (int j = max(0, issued - STAGES); j < issued; ++j) dec_wait_drain(&bk->full[j % STAGES], (j / STAGES) & 1);
+      for (int j = max(0, issued - STAGES + (drained_marker ? 1 : 0)); j < issued; ++j)
+        dec_wait_drain(&bk->full[j % STAGES], (j / STAGES) & 1);
     __syncwarp();
   } else if (warp == kDecMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -283,9 +418,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mma_commit(&bk->empty[j % STAGES]);
         return true;
       };
-      for (int it = 0; it < n_it && ok; ++it) {
+      for (int it = 0; ok; ++it) {
         const int s = it % STAGES, sb = it & 1;
         if (!mbar_wait(&bk->full[s], (it / STAGES) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
+        if (bk->stage_tile[s] < 0) {
+          // end marker: finish the last tile, then release the softmax warps
+          if (it > 0) ok = issue_pv(it - 1);
+          n_it = it;
+          mbar_arrive(&bk->s_full[sb]);
+          break;
+        }
         if (it >= 2 && !mbar_wait(&bk->s_free[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
           break;
         tc_fence_after();
@@ -299,7 +441,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mma_commit(&bk->s_full[sb]);
         if (it > 0) ok = issue_pv(it - 1);
       }
-      if (ok && n_it > 0 && !*abort_flag) issue_pv(n_it - 1);
       mma_commit(&bk->drain);
       dec_wait_drain(&bk->drain, 0);
     }
@@ -313,14 +454,24 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
     for (int q = 0; q < NQ; ++q)
       if (q < n_rows && (q % a.qcap) < nq_b) qvalid |= (1ull << q);
-    // A warp whose wait ran out keeps iterating without waits or tensor-memory access, so
-    // that all four warps execute the same sequence of named-barrier operations.
+    // The loop ends, in all four warps at once, at the end marker or when a wait ran out.
+    // A warp whose wait ran out inside an iteration finishes it without waits or
+    // tensor-memory access, so that all four warps take the same named-barrier steps.
     bool ok = true;
-    for (int it = 0; it < n_it; ++it) {
+    int it = 0;
+    for (;; ++it) {
       const int sb = it & 1;
       if (ok)
         ok = __all_sync(0xffffffffu,
                         mbar_wait(&bk->s_full[sb], (it >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_SOFTMAX));
+      int tile = -1;
+      if (ok) {
+        // the stage's tile id, published by the producer before it completed full[stage]
+        ok = __all_sync(0xffffffffu, mbar_wait(&bk->full[it % STAGES], (it / STAGES) & 1, abort_flag, a.dev_err,
+                                               DEV_ERR_TIMEOUT_SOFTMAX));
+        if (ok) tile = bk->stage_tile[it % STAGES];
+      }
+      if (bar_red_or(1, 128, tile < 0 || *abort_flag != 0)) break;
       float sv[NQ];
 #pragma unroll
       for (int q = 0; q < NQ; ++q) sv[q] = 0.f;
@@ -338,7 +489,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bk->s_free[sb]);
-      const bool kv = ok && slot_valid<SPARSE>(sl, a.L, a.bs, G, (t_begin + it) * 128 + t);
+      const bool kv = ok && slot_valid<SPARSE>(sl, a.L, a.bs, G, tile * 128 + t);
       bool over = false;
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
@@ -417,6 +568,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bk->p_full[sb]);
     }
+    n_it = it;
     if (ok && n_it > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bk->pv_done[(n_it - 1) & 1], ((n_it - 1) >> 1) & 1, abort_flag,
                                              a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE));
@@ -581,7 +733,7 @@ int dec_make_map(CUtensorMap* map, const void* base, int BH, int L, int box_rows
   return FOCUS_OK;
 }
 
-template <int NQ, int STAGES, bool SPARSE>
+template <int NQ, int STAGES, bool SPARSE, bool FUSED>
 int max_active_clusters(int cs) {
   static std::mutex mu;
   static std::map<std::pair<int, int>, int> cache;
@@ -591,7 +743,7 @@ int max_active_clusters(int cs) {
   auto key = std::make_pair(dev, cs);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE>;
+  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(DecSmem<NQ, STAGES>::kBytes));
   cudaLaunchConfig_t cfg = {};
@@ -614,17 +766,17 @@ int max_active_clusters(int cs) {
   return n;
 }
 
-template <int NQ, int STAGES, bool SPARSE>
+template <int NQ, int STAGES, bool SPARSE, bool FUSED>
 int choose_cluster(int units) {
   const int sms = device_sm_count();
   for (int cs : {8, 4, 2}) {
     if (units * cs > sms) continue;
-    if (max_active_clusters<NQ, STAGES, SPARSE>(cs) >= units) return cs;
+    if (max_active_clusters<NQ, STAGES, SPARSE, FUSED>(cs) >= units) return cs;
   }
   return 1;
 }
 
-template <int NQ, int STAGES, bool SPARSE>
+template <int NQ, int STAGES, bool SPARSE, bool FUSED>
 int run_decode(const DecArgs& a0, cudaStream_t stream) {
   DecArgs a = a0;
   CUtensorMap mk, mv;
@@ -634,8 +786,8 @@ int run_decode(const DecArgs& a0, cudaStream_t stream) {
   if (st != FOCUS_OK) return st;
   a.dev_err = device_error_word();
   const int units = a.B * a.Hkv;
-  const int cs = choose_cluster<NQ, STAGES, SPARSE>(units);
-  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE>;
+  const int cs = choose_cluster<NQ, STAGES, SPARSE, FUSED>(units);
+  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        static_cast<int>(DecSmem<NQ, STAGES>::kBytes));
   const cudaError_t e =
@@ -661,10 +813,15 @@ bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C) {
   return d == kDecD && (Hq / Hkv) * qcap <= 64 && L >= 8 && S <= kDecMaxSinks && C <= kDecMaxBlocks;
 }
 
+// Fused relevance + top-C is used when kbar is given (blocks is then ignored).
+bool decode_fused_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C, int nb) {
+  return decode_supported(d, Hq, Hkv, qcap, L, S, C) && nb >= 1 && nb <= kDecMaxNb;
+}
+
 int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                      __nv_bfloat16* O, float* lse_out, const int32_t* sinks, const int32_t* blocks, int S, int C, int bs,
                      int P, int g0, int g1, bool sparse, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, const float* kbar, int nb, int32_t* blocks_out) {
   DecArgs a{};
   a.Q = Q;
   a.n_q = n_q;
@@ -698,9 +855,15 @@ int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bflo
     a.gen_pad = 0;
   }
   const int nrows = a.g * qcap;
+  if (kbar) {
+    a.kbar = kbar;
+    a.nb = nb;
+    a.blocks_out = blocks_out;
+    return nrows <= 32 ? run_decode<32, 3, true, true>(a, stream) : run_decode<64, 2, true, true>(a, stream);
+  }
   if (nrows <= 32)
-    return sparse ? run_decode<32, 3, true>(a, stream) : run_decode<32, 3, false>(a, stream);
-  return sparse ? run_decode<64, 2, true>(a, stream) : run_decode<64, 2, false>(a, stream);
+    return sparse ? run_decode<32, 3, true, false>(a, stream) : run_decode<32, 3, false, false>(a, stream);
+  return sparse ? run_decode<64, 2, true, false>(a, stream) : run_decode<64, 2, false, false>(a, stream);
 }
 
 }  // namespace focus

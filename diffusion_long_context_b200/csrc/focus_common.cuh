@@ -209,6 +209,21 @@ __device__ __forceinline__ uint32_t dsmem_addr(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
+// Split cluster barrier: arrive early, wait later (every thread of every CTA does both,
+// with no other cluster barrier in between).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// Atomic add on a 32-bit word of CTA `rank`'s shared memory; returns the old value.
+__device__ __forceinline__ uint32_t dsmem_atomic_add(uint32_t local_saddr, uint32_t rank, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.shared::cluster.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(dsmem_addr(local_saddr, rank)), "r"(v)
+               : "memory");
+  return old;
+}
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");

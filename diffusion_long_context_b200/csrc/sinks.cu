@@ -10,7 +10,8 @@
 
 namespace focus {
 
-// The L column sums of (b, h) are staged in shared memory when they fit (STAGE = true).
+// The L column sums of (b, h) are staged in shared memory, as order keys, when they fit
+// (STAGE = true); the block-wide radix selection then reads shared memory only.
 template <bool STAGE>
 __global__ void __launch_bounds__(1024) sink_topk_kernel(const float* __restrict__ colsum, int L, int S,
                                                          int32_t* __restrict__ sinks) {
@@ -20,19 +21,22 @@ __global__ void __launch_bounds__(1024) sink_topk_kernel(const float* __restrict
   __shared__ TopkShared tk;
   const int bh = blockIdx.x;
   const float* row = colsum + static_cast<size_t>(bh) * L;
+  int32_t* out = sinks + static_cast<size_t>(bh) * S;
   if (STAGE) {
+    uint32_t* s_key = reinterpret_cast<uint32_t*>(s_row);
     if ((L & 3) == 0) {
-      for (int i = threadIdx.x; i < L / 4; i += blockDim.x)
-        reinterpret_cast<float4*>(s_row)[i] = __ldg(reinterpret_cast<const float4*>(row) + i);
+      for (int i = threadIdx.x; i < L / 4; i += blockDim.x) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(row) + i);
+        reinterpret_cast<uint4*>(s_key)[i] =
+            make_uint4(float_order_key(v.x), float_order_key(v.y), float_order_key(v.z), float_order_key(v.w));
+      }
     } else {
-      for (int i = threadIdx.x; i < L; i += blockDim.x) s_row[i] = __ldg(row + i);
+      for (int i = threadIdx.x; i < L; i += blockDim.x) s_key[i] = float_order_key(__ldg(row + i));
     }
     __syncthreads();
-    block_topk_ascending([&](int i) { return float_order_key(s_row[i]); }, L, S,
-                         sinks + static_cast<size_t>(bh) * S, S, tk);
+    block_topk_ascending([&](int i) { return s_key[i]; }, L, S, out, S, tk);
   } else {
-    block_topk_ascending([&](int i) { return float_order_key(__ldg(row + i)); }, L, S,
-                         sinks + static_cast<size_t>(bh) * S, S, tk);
+    block_topk_ascending([&](int i) { return float_order_key(__ldg(row + i)); }, L, S, out, S, tk);
   }
 }
 

@@ -36,10 +36,14 @@ __device__ __forceinline__ SlotLayout build_sparse_layout(const int32_t* blk_g, 
                                                           int max_blocks, int* s_sinks, int max_sinks,
                                                           SlotLayout* out) {
   const int lane = threadIdx.x & 31;
+  // the first 64 block entries and 32 sinks are fetched together (one memory round trip)
+  const int pre_b0 = (lane < C) ? blk_g[lane] : -1;
+  const int pre_b1 = (32 + lane < C) ? blk_g[32 + lane] : -1;
+  const int pre_s0 = (lane < S) ? snk_g[lane] : -1;
   int nvb = 0;
   for (int i0 = 0; i0 < C; i0 += 32) {
     const int i = i0 + lane;
-    const int v = (i < C) ? blk_g[i] : -1;
+    const int v = i0 == 0 ? pre_b0 : i0 == 32 ? pre_b1 : ((i < C) ? blk_g[i] : -1);
     const unsigned m = __ballot_sync(0xffffffffu, v >= 0);
     if (v >= 0 && i < max_blocks) s_blk[i] = v;
     nvb += __popc(m);
@@ -52,7 +56,7 @@ __device__ __forceinline__ SlotLayout build_sparse_layout(const int32_t* blk_g, 
   int nf = 0, prev_last = -1;
   for (int i0 = 0; i0 < S; i0 += 32) {
     const int i = i0 + lane;
-    const int j = (i < S) ? snk_g[i] : -1;
+    const int j = i0 == 0 ? pre_s0 : ((i < S) ? snk_g[i] : -1);
     const int jprev = __shfl_up_sync(0xffffffffu, j, 1);
     const int before = (lane == 0) ? prev_last : jprev;
     bool keep = (j >= 0) && (j < L) && !(j >= g0 && j < g1) && (j != before);

@@ -47,6 +47,8 @@ _SIGS = {
     "focus_sparse_workspace_bytes": (_sz, [_i] * 12),
     "focus_sparse_attention_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
                                             _i, _f, _p, _p]),
+    "focus_sparse_attention_fused": (_i, [_p, _p, _p, _p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+                                          _i, _f, _p, _p, _p, _sz, _p]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -219,3 +221,28 @@ def focus_sparse_attention(Q_active, n_active, K, V, sinks, blocks, bs, P, g0, g
                                     _ptr(blocks), C, bs, P, g0, g1, B, Hq, Hkv, L, d, acap, float(scale),
                                     _ptr(O_active), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "focus_sparse_attention")
+
+
+def focus_sparse_attention_fused(Q_active, n_active, K, V, kbar, C, sinks, bs, P, g0, g1, blocks, O_active, scale=None,
+                                 ws=None, stream=None):
+    """Block relevance + top-C + sparse attention of one layer (blocks receives the kept blocks)."""
+    _need(Q_active, torch.bfloat16, "Q_active", 4)
+    _need(n_active, torch.int32, "n_active", 1)
+    _need(K, torch.bfloat16, "K", 4)
+    _need(V, torch.bfloat16, "V", 4)
+    _need(kbar, torch.float32, "kbar", 4)
+    _need(blocks, torch.int32, "blocks", 3)
+    _need(O_active, torch.bfloat16, "O_active", 4)
+    if sinks is not None:
+        _need(sinks, torch.int32, "sinks", 3)
+    B, Hq, acap, d = Q_active.shape
+    Hkv, L = K.shape[1], K.shape[2]
+    nb = kbar.shape[2]
+    S = 0 if sinks is None else sinks.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = sparse_workspace_bytes(B, Hq, Hkv, L, d, acap, S, C, bs, P, g0, g1)
+    ws, ws_bytes = _workspace(need, Q_active.device, ws)
+    st = lib.focus_sparse_attention_fused(_ptr(Q_active), _ptr(n_active), _ptr(K), _ptr(V), _ptr(kbar), nb, C,
+                                          _ptr(sinks), S, bs, P, g0, g1, B, Hq, Hkv, L, d, acap, float(scale),
+                                          _ptr(blocks), _ptr(O_active), _ptr(ws), ws_bytes, _stream(stream))
+    _check(st, "focus_sparse_attention_fused")

@@ -3,7 +3,7 @@
 A non-block-entry step (Focus-dLLM summary page, "方法步骤详情" / method steps (1)-(5)):
   select_queries -> gather the active query rows of every layer -> layers 0..l_dense:
   dense attention (layer l_dense also produces the sink column sums) -> sink top-S ->
-  layers > l_dense: block relevance + top-C, sparse attention over sinks U blocks U
+  layers > l_dense: block relevance + top-C, then sparse attention over sinks U blocks U
   current block.
 A block-entry step refreshes the block means of every sparse layer (and, for the
 comparison, runs the dense full refresh).
@@ -95,6 +95,13 @@ class SparseStep:
         F.focus_sparse_attention(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.sinks,
                                  self.blocks[l], c.bs, c.P, c.g0, c.g1, self.O_active[l], scale=self.scale,
                                  ws=self.ws)
+
+    def sparse_layer_fused(self, l: int):
+        """Block relevance + top-C + sparse attention of layer l in one launch."""
+        c = self.cfg
+        F.focus_sparse_attention_fused(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.kbar[l], c.C,
+                                       self.sinks, c.bs, c.P, c.g0, c.g1, self.blocks[l], self.O_active[l],
+                                       scale=self.scale, ws=self.ws)
 
     def run(self, timers=None):
         """Eager step. `timers` (optional) maps a call kind to a list receiving (start, end) events."""

@@ -169,6 +169,21 @@ FOCUS_API int focus_sparse_attention(const focus_bf16* Q_active, const int32_t* 
                            int P, int g0, int g1, int B, int Hq, int Hkv, int L, int d, int acap, float scale,
                            focus_bf16* O_active, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * (4b)+(5) Block relevance, top-C and sparse attention of one layer in a single launch --
+ * method steps (4) and (5). Same results as focus_block_select (kept blocks written to
+ * blocks [B, Hkv, C], -1 tail) followed by focus_sparse_attention on them. kbar
+ * [B, Hkv, nb, d] fp32 with nb = ceil(P / bs). Shapes outside the fused kernel's range
+ * (d != 128, more than 64 query rows per KV head, nb > 4096, C > 512 or S > 512) run the
+ * two calls in sequence; ws/ws_bytes then serve focus_sparse_attention (size them with
+ * focus_sparse_workspace_bytes).
+ */
+FOCUS_API int focus_sparse_attention_fused(const focus_bf16* Q_active, const int32_t* n_active, const focus_bf16* K,
+                                           const focus_bf16* V, const float* kbar, int nb, int C,
+                                           const int32_t* sinks, int S, int bs, int P, int g0, int g1, int B, int Hq,
+                                           int Hkv, int L, int d, int acap, float scale, int32_t* blocks,
+                                           focus_bf16* O_active, void* ws, size_t ws_bytes, void* stream);
+
 FOCUS_API size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int acap, int S, int C, int bs, int P,
                                     int g0, int g1);
 

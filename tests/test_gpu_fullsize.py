@@ -57,7 +57,12 @@ def _run_two_layers(F, cfg):
             blocks = torch.empty((cfg.B, cfg.Hkv, cfg.C), **i32)
             F.focus_block_select(Qa, n_active, kbar, cfg.C, blocks)
             F.focus_sparse_attention(Qa, n_active, K, V, out["sinks"], blocks, cfg.bs, cfg.P, cfg.g0, cfg.g1, O)
-            out.update(kbar=kbar, blocks=blocks)
+            # the fused single-launch layer (the step's path) must agree with the two calls
+            blocks_f = torch.empty_like(blocks)
+            O_f = torch.empty_like(O)
+            F.focus_sparse_attention_fused(Qa, n_active, K, V, kbar, cfg.C, out["sinks"], cfg.bs, cfg.P, cfg.g0,
+                                           cfg.g1, blocks_f, O_f)
+            out.update(kbar=kbar, blocks=blocks, blocks_fused=blocks_f, O_fused=O_f)
         out["O_" + tag] = O
     torch.cuda.synchronize()
     assert F.device_error() == 0
@@ -108,6 +113,8 @@ def _check_against_oracle(cfg, st, lay_d, lay_s, i_focus, i_active, out):
         f"{cfg.name}: {sink_ties} sink / {block_ties} block near-tie sets (valid, but not bit-exact)"
     Os = orc.sparse_attention(Qa, nA, Ks, Vs, sinks, blocks, cfg.bs, cfg.P, cfg.g0, cfg.g1, scale)
     assert_attention_close(out["O_sparse"], Os, rows_valid=nA, what=f"{cfg.name} sparse layer")
+    assert torch.equal(out["blocks_fused"], out["blocks"]), f"{cfg.name}: fused top-C differs"
+    assert_attention_close(out["O_fused"], Os, rows_valid=nA, what=f"{cfg.name} fused sparse layer")
 
 
 @pytest.mark.parametrize("cfg", [configs.LLADA_8K, configs.DREAM_16K, configs.FULL_32K],

@@ -371,3 +371,49 @@ def test_composed_step_small(F):
             assert np.array_equal(blocks_all[l].cpu().numpy(), ref["blocks"][l]), f"layer {l} blocks differ"
         assert_attention_close(outs[l], ref["O"][l], rows_valid=nA, what=f"layer {l}")
     assert F.device_error() == 0
+
+
+# ------------------------------------------------------------------ fused relevance + top-C + sparse attention
+FUSED_CASES = [
+    # name, B, Hq, Hkv, P, G, L, bs, C, S, acap, n_active
+    ("mha_bs64", 1, 4, 4, 2048, 32, 2112, 64, 8, 8, 32, [30]),
+    ("mha_b2_bs32", 2, 4, 4, 1024, 32, 1088, 32, 12, 16, 32, [32, 9]),
+    ("gqa2", 1, 8, 4, 1500, 32, 1600, 64, 5, 6, 32, [27]),
+    ("ragged_bs24", 1, 2, 2, 250, 20, 300, 24, 4, 3, 20, [20]),
+    ("gqa7_fallback", 1, 28, 4, 1024, 32, 1100, 64, 6, 8, 32, [31]),     # 224 rows: two-call path
+]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES, ids=[c[0] for c in FUSED_CASES])
+def test_sparse_fused_matches_oracle_and_two_calls(F, case):
+    name, B, Hq, Hkv, P, G, L, bs, C, S, acap, n_act = case
+    g0, g1 = P, P + G
+    d = 128
+    rng = np.random.default_rng(len(name) + L)
+    Q = inputs.random_bf16((B, Hq, acap, d), seed=L + 31, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=L + 32, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=L + 33, device=DEV)
+    n_active = torch.tensor(n_act, dtype=torch.int32, device=DEV)
+    nb = -(-P // bs)
+    kbar = torch.empty((B, Hkv, nb, d), dtype=torch.float32, device=DEV)
+    F.focus_block_means(K, P, bs, kbar)
+    sinks = torch.from_numpy(np.sort(np.stack([np.stack([rng.choice(L, S, replace=False) for _ in range(Hkv)])
+                                                for _ in range(B)]), axis=-1).astype(np.int32)).to(DEV)
+    blocks_f = _i32((B, Hkv, C))
+    O_f = torch.full((B, Hq, acap, d), 4.0, dtype=torch.bfloat16, device=DEV)
+    F.focus_sparse_attention_fused(Q, n_active, K, V, kbar, C, sinks, bs, P, g0, g1, blocks_f, O_f)
+    blocks_2 = _i32((B, Hkv, C))
+    O_2 = torch.full((B, Hq, acap, d), 4.0, dtype=torch.bfloat16, device=DEV)
+    F.focus_block_select(Q, n_active, kbar, C, blocks_2)
+    F.focus_sparse_attention(Q, n_active, K, V, sinks, blocks_2, bs, P, g0, g1, O_2)
+    torch.cuda.synchronize()
+    assert torch.equal(blocks_f, blocks_2), "fused top-C differs from focus_block_select"
+    # oracle: its own block means and relevance from the same inputs
+    Q64, K64, V64 = inputs.to_f64(Q), inputs.to_f64(K), inputs.to_f64(V)
+    ref_blocks, R = orc.block_select(Q64, n_act, orc.block_means(K64, P, bs), C)
+    assert np.array_equal(blocks_f.cpu().numpy(), ref_blocks), "kept blocks differ from the oracle"
+    ref = orc.sparse_attention(Q64, n_act, K64, V64, sinks.cpu().numpy(), ref_blocks, bs, P, g0, g1,
+                               float(np.float32(1 / math.sqrt(d))))
+    assert_attention_close(O_f, ref, rows_valid=n_act, what=f"fused sparse ({name})")
+    assert (O_f.float() - O_2.float()).abs().max().item() <= 1e-2
+    assert F.device_error() == 0
