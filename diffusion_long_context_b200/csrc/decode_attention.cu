@@ -78,6 +78,7 @@ struct __align__(8) DecBook {
   int blk[kDecMaxBlocks];
   int sinks[kDecMaxSinks];
   TopkShared tk;
+  uint32_t qvalid[2];      // bit q: query column q is a real query
   uint32_t tile_ctr;       // next dynamically claimed tile (CTA 0 of the cluster)
   int stage_tile[4];       // tile held by each ring stage, -1 = no more tiles
 };
@@ -131,6 +132,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int nq_b = a.n_q ? min(a.n_q[b], a.qcap) : a.qcap;
   const int n_rows = a.g * a.qcap;             // <= NQ
   const int G = a.g1 - a.g0;
+  FastDiv qdiv;                                // query column q <-> (head q / qcap, row q % qcap)
+  qdiv.init(static_cast<uint32_t>(a.qcap), 64u);
 
   // ---------------------------------------------------------------- prologue
   // The producer warp initialises the barriers, builds the slot layout and issues the first
@@ -142,6 +145,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const __nv_bfloat16* Kbh = a.K + static_cast<size_t>(bh) * a.L * D;
   const __nv_bfloat16* Vbh = a.V + static_cast<size_t>(bh) * a.L * D;
   int issued = 0;
+  const uint64_t l2_stream = l2_evict_first_policy();   // K/V rows are read once per call
   SlotLayout sl_p{};
   int p_n = 0;                 // tiles of this (b, h)
   bool p_more = true;          // the end marker is not issued yet
@@ -163,8 +167,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int k0 = group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + grp * BR);
       const int at = (j >> 1) & 1;
       const uint32_t off = at * (128 * 128) + grp * BR * 128;
-      if (j & 1) tma_load_3d(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, k0, bh);
-      else tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh);
+      if (j & 1) tma_load_3d_hint(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, k0, bh, l2_stream);
+      else tma_load_3d_hint(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh, l2_stream);
     }
     if (SPARSE && tma_mask != all_groups) {
       // sink rows (and rows past the end, zero-filled) by cp.async, 16 bytes per lane
@@ -338,7 +342,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int q = idx / CH, c = idx % CH;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (q < n_rows) {
-        const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
+        const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
+        const int hq = kvh * a.g + qh, i = q - qh * a.qcap;
         v = __ldg(reinterpret_cast<const uint4*>(a.Q + ((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D) + c);
         if (i >= nq_b) v = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -347,6 +352,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (threadIdx.x < NQ) {
       bk->mref[threadIdx.x] = -INFINITY;
       bk->alpha[threadIdx.x] = 1.f;
+    }
+    if (warp < 2) {
+      const int q = threadIdx.x;
+      const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
+      const unsigned m = __ballot_sync(0xffffffffu, q < NQ && q < n_rows && (q - qh * a.qcap) < nq_b);
+      if (lane == 0) bk->qvalid[warp] = m;
     }
     fence_proxy_async_smem();
   }
@@ -450,10 +461,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int t = threadIdx.x;                         // key of the tile == TMEM lane == dim of O^T
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tO = tmem + 2 * NQ;
-    uint64_t qvalid = 0;                               // bit q: query column q is a real query
-#pragma unroll
-    for (int q = 0; q < NQ; ++q)
-      if (q < n_rows && (q % a.qcap) < nq_b) qvalid |= (1ull << q);
+    const uint64_t qvalid = bk->qvalid[0] | (static_cast<uint64_t>(bk->qvalid[1]) << 32);
     // The loop ends, in all four warps at once, at the end marker or when a wait ran out.
     // A warp whose wait ran out inside an iteration finishes it without waits or
     // tensor-memory access, so that all four warps take the same named-barrier steps.
@@ -498,16 +506,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       if (bar_red_or(1, 128, over)) {
         // exact per-query maximum of this tile, then move the references up
+        // (one redux per query on the order-preserving integer image of the score)
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
-          float m = sv[q];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-          if (lane == 0) bk->red[warp][q] = m;
+          const uint32_t m = __reduce_max_sync(0xffffffffu, float_order_key(sv[q]));
+          if (lane == 0) bk->red[warp][q] = __uint_as_float(m);
         }
         named_bar_sync(1, 128);
         if (t < NQ) {
-          const float mt = fmaxf(fmaxf(bk->red[0][t], bk->red[1][t]), fmaxf(bk->red[2][t], bk->red[3][t]));
+          const uint32_t k01 = max(__float_as_uint(bk->red[0][t]), __float_as_uint(bk->red[1][t]));
+          const uint32_t k23 = max(__float_as_uint(bk->red[2][t]), __float_as_uint(bk->red[3][t]));
+          const float mt = order_key_to_float(max(k01, k23));
           const float mo = bk->mref[t];
           const float mn = fmaxf(mo, mt);
           if (mn > mo + 8.f || (mo == -INFINITY && mn > -INFINITY)) {
@@ -574,35 +583,29 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                              a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE));
       tc_fence_after();
     }
-    // row sums: reduce the per-key partials over the 128 threads
+    // row sums: reduce the per-key partials over the 128 threads (reduce-scatter per warp,
+    // then the four warps' sums; the epilogue's CTA barrier orders lfin)
+    warp_sum_scatter<NQ>(lsum);
 #pragma unroll
-    for (int q = 0; q < NQ; ++q) {
-      float v = lsum[q];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) bk->red[warp][q] = v;
-    }
+    for (int j = 0; j < NQ / 32; ++j) bk->red[warp][lane * (NQ / 32) + j] = lsum[j];
     named_bar_sync(1, 128);
     if (t < NQ) bk->lfin[t] = (bk->red[0][t] + bk->red[1][t]) + (bk->red[2][t] + bk->red[3][t]);
-    named_bar_sync(1, 128);
     if (!ok) bk->abort_flag = 1;
   }
 
   // ---------------------------------------------------------------- epilogue
-  // Query q is finalised by CTA q % cs of the cluster. Every CTA pushes its partial row of
-  // q (m, l and the unnormalised O row) into the owner's receive buffer with DSMEM stores;
-  // two cluster barriers frame the pushes, and the owner merges from its own memory.
-  // Receive buffer (in the V ring, idle once every CTA of the cluster is past the first
-  // barrier): recv_o[q / cs][src][D], recv_ml[q / cs][src][2].
+  // Every CTA leaves its partial result (unnormalised O^T, m and l of every query) in its
+  // own V ring, idle once its loop is done. After one cluster barrier, CTA r merges the
+  // queries [r * qpc, (r + 1) * qpc) from the partials of all CTAs of the cluster, read over
+  // distributed shared memory with 16-byte loads; a split barrier (arrive after the reads,
+  // wait before exit) keeps every CTA's partials resident until all readers are done.
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const bool have_o = (n_it > 0) && !bk->abort_flag;
-  // index (q / cs) * cs + src < NQ + cs <= NQ + 8: (NQ + 8) x D floats fit in the V ring
-  static_assert((NQ + 8) * (D + 2) * 4 + NQ * 8 * 4 <= STAGES * SM::kTile, "receive buffer exceeds the V ring");
-  float* recv_o = reinterpret_cast<float*>(sV);    // [(q / cs) * cs + src][D]
-  float* recv_ml = recv_o + (NQ + 8) * D;          // [(q / cs) * cs + src][2]
-  float ov[NQ];
+  static_assert(NQ * D * 4 + NQ * 8 <= STAGES * SM::kTile, "partials exceed the V ring");
+  float* part_o = reinterpret_cast<float*>(sV);                      // [NQ][D]
+  float2* part_ml = reinterpret_cast<float2*>(part_o + NQ * D);      // [NQ] (m, l)
   if (warp < 4) {
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
 #pragma unroll
@@ -615,88 +618,72 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         tmem_ld_wait();
       }
 #pragma unroll
-      for (int j = 0; j < 32; ++j) ov[c * 32 + j] = __uint_as_float(rg[j]);
+      for (int j = 0; j < 32; ++j) part_o[(c * 32 + j) * D + threadIdx.x] = __uint_as_float(rg[j]);
     }
-  }
-  if (cs > 1) cluster_sync();        // every CTA of the cluster is done with its rings
-  else __syncthreads();
-  if (warp < 4) {
-    const int t = threadIdx.x;
-    const uint32_t ro_s = smem_u32(recv_o), rml_s = smem_u32(recv_ml);
-#pragma unroll
-    for (int q = 0; q < NQ; ++q) {
-      if (q >= n_rows) break;
-      const int owner = q % cs, slot = q / cs;
-      const uint32_t off = static_cast<uint32_t>(((slot * cs + rank) * D + t) * 4);
-      if (cs > 1) {
-        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_addr(ro_s + off, owner)), "f"(ov[q]) : "memory");
-      } else {
-        recv_o[(slot * cs + rank) * D + t] = ov[q];
-      }
-    }
-    if (t < n_rows) {
-      const int q = t, owner = q % cs, slot = q / cs;
-      const uint32_t off = static_cast<uint32_t>(((slot * cs + rank) * 2) * 4);
-      const float mq = bk->mref[q], lq = have_o ? bk->lfin[q] : 0.f;
-      if (cs > 1) {
-        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_addr(rml_s + off, owner)), "f"(mq) : "memory");
-        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(dsmem_addr(rml_s + off + 4, owner)), "f"(lq) : "memory");
-      } else {
-        recv_ml[(slot * cs + rank) * 2] = mq;
-        recv_ml[(slot * cs + rank) * 2 + 1] = lq;
-      }
-    }
-  }
-  if (cs > 1) cluster_sync();        // pushes visible to their owners
-  else __syncthreads();
-  // per-query merge weights, one thread per owned query: w[src] = 2^(m_src - M) / l
-  float* mw = recv_ml + (NQ + 8) * 2;            // [owned query][8] weights
-  if (warp < 4) {
-    const int t = threadIdx.x;
-    const int q = rank + t * cs;
-    if (q < n_rows) {
-      const int slot = q / cs;
-      float M = -INFINITY;
-      for (int r = 0; r < cs; ++r)
-        if (recv_ml[(slot * cs + r) * 2 + 1] > 0.f) M = fmaxf(M, recv_ml[(slot * cs + r) * 2]);
-      float l = 0.f;
-      float w[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        w[r] = 0.f;
-        if (r < cs && M > -INFINITY) {
-          const float lr = recv_ml[(slot * cs + r) * 2 + 1];
-          if (lr > 0.f) {
-            w[r] = exp2_approx(recv_ml[(slot * cs + r) * 2] - M);
-            l += w[r] * lr;
-          }
-        }
-      }
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (r < cs) mw[t * 8 + r] = w[r] * inv;
-      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
-      if (a.lse_out && i < nq_b) a.lse_out[(static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i] = M + __log2f(l);
-    }
-    named_bar_sync(1, 128);
-    for (int qi = 0, q = rank; q < n_rows; ++qi, q += cs) {
-      const int slot = q / cs;
-      const int hq = kvh * a.g + q / a.qcap, i = q % a.qcap;
-      float o = 0.f;
-      if (i < nq_b)
-        for (int r = 0; r < cs; ++r) o += mw[qi * 8 + r] * recv_o[(slot * cs + r) * D + t];
-      a.O[((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D + t] = __float2bfloat16_rn(o);
-    }
+    if (threadIdx.x < NQ)
+      part_ml[threadIdx.x] = make_float2(bk->mref[threadIdx.x], have_o ? bk->lfin[threadIdx.x] : 0.f);
   }
   tc_fence_before();
-  __syncthreads();
+  if (cs > 1) cluster_sync();        // every partial of the cluster is in place
+  else __syncthreads();
   if (warp == kDecMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, SM::kTmemCols);
   }
+  const int qpc = (n_rows + cs - 1) / cs;
+  if (warp < 4) {
+    // lane: dims 4*lane .. 4*lane+3; warp: queries rank*qpc + warp + 4k
+    const uint32_t po = smem_u32(part_o), pm = smem_u32(part_ml);
+    for (int qi = warp; qi < qpc; qi += 4) {
+      const int q = rank * qpc + qi;
+      if (q >= n_rows) break;
+      float4 ov[8];
+      float2 ml[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        ov[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        ml[r] = make_float2(-INFINITY, 0.f);
+        if (r < cs) {
+          ml[r] = dsmem_ld_v2(dsmem_addr(pm + static_cast<uint32_t>(q) * 8u, r));
+          ov[r] = dsmem_ld_v4(dsmem_addr(po + static_cast<uint32_t>(q * D + 4 * lane) * 4u, r));
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (ml[r].y > 0.f) M = fmaxf(M, ml[r].x);
+      float l = 0.f, w[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        w[r] = ml[r].y > 0.f ? exp2_approx(ml[r].x - M) : 0.f;
+        l += w[r] * ml[r].y;
+      }
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float wr = w[r] * inv;
+        o.x += wr * ov[r].x;
+        o.y += wr * ov[r].y;
+        o.z += wr * ov[r].z;
+        o.w += wr * ov[r].w;
+      }
+      const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
+      const int hq = kvh * a.g + qh, i = q - qh * a.qcap;
+      if (i >= nq_b) o = make_float4(0.f, 0.f, 0.f, 0.f);
+      uint2 pk;
+      pk.x = pack_bf16x2(o.x, o.y);
+      pk.y = pack_bf16x2(o.z, o.w);
+      const size_t row = (static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i;
+      *reinterpret_cast<uint2*>(a.O + row * D + 4 * lane) = pk;
+      if (lane == 0 && a.lse_out && i < nq_b) a.lse_out[row] = M + __log2f(l);
+    }
+  }
+  if (cs > 1) {
+    cluster_arrive();                // this CTA's reads of the partials are done
+    cluster_wait();                  // no CTA leaves while its partials may still be read
+  }
 }
-
 // ------------------------------------------------------------------------- host side
 namespace {
 

@@ -99,6 +99,20 @@ cudaError_t launch_k_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, si
 // ------------------------------------------------------------------ device side
 #if defined(__CUDACC__)
 
+// Exact unsigned division by a divisor fixed per CTA. When every dividend n satisfies
+// n * d < 2^32, floor(n / d) = umulhi(n, m) with m = ceil(2^32 / d) (Granlund & Montgomery,
+// "Division by invariant integers using multiplication", 1994); otherwise a plain division.
+struct FastDiv {
+  uint32_t d, m;
+  __host__ __device__ void init(uint32_t dd, uint32_t n_max) {
+    d = dd;
+    m = (dd > 1 && static_cast<unsigned long long>(n_max) * dd < (1ull << 32))
+            ? static_cast<uint32_t>(0xFFFFFFFFull / dd + 1ull)
+            : 0u;
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const { return m ? __umulhi(n, m) : (d == 1 ? n : n / d); }
+};
+
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -188,6 +202,22 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Same, with an L2 cache policy (from l2_evict_first_policy) for data read once.
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                                 int z, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cta.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
+      "%4, %5}], [%2], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+// L2 policy: lines fetched under it are the first to be evicted (streamed K/V).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // ---- cp.async (16 bytes; src_bytes = 0 writes zeros without reading)
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -223,6 +253,19 @@ __device__ __forceinline__ uint32_t dsmem_atomic_add(uint32_t local_saddr, uint3
                : "r"(dsmem_addr(local_saddr, rank)), "r"(v)
                : "memory");
   return old;
+}
+__device__ __forceinline__ float4 dsmem_ld_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ float2 dsmem_ld_v2(uint32_t addr) {
+  float2 v;
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  return v;
 }
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
   float v;
@@ -353,6 +396,29 @@ __device__ __forceinline__ uint32_t float_order_key(float f) {
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inverse of float_order_key.
+__device__ __forceinline__ float order_key_to_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Warp reduce-scatter of N per-lane values (N a multiple of 32): afterwards v[j] of lane
+// l, j < N / 32, holds the sum over the 32 lanes of value index l * (N / 32) + j.
+// 31 * N / 32 shuffles instead of 5 * N for N separate butterfly sums.
+template <int N>
+__device__ __forceinline__ void warp_sum_scatter(float (&v)[N]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 16, w = N / 2; off >= 1; off >>= 1, w >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int j = 0; j < w; ++j) {
+      const float send = upper ? v[j] : v[j + w];
+      const float keep = upper ? v[j + w] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
 }
 
 #endif  // __CUDACC__

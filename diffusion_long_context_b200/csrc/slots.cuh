@@ -24,6 +24,7 @@ struct SlotLayout {
   int nvb;          // kept blocks (valid entries of the block list)
   int last_size;    // valid keys of the last kept block (short when it ends at P)
   int n_fsinks;     // sinks that remain after de-duplication
+  FastDiv pad_div;  // division by pad_bs for any slot below n_slots + 128
 };
 
 // One warp builds the layout of (b, h): copies the kept-block list to s_blk (up to
@@ -88,6 +89,7 @@ __device__ __forceinline__ SlotLayout build_sparse_layout(const int32_t* blk_g, 
   sl.sink_start = sl.gen_start + gen_pad;
   sl.n_fsinks = min(nf, max_sinks);
   sl.n_slots = sl.sink_start + sl.n_fsinks;
+  sl.pad_div.init(static_cast<uint32_t>(sl.pad_bs), static_cast<uint32_t>(sl.n_slots + 128));
   if (lane == 0) *out = sl;
   return sl;
 }
@@ -98,7 +100,7 @@ template <bool SPARSE>
 __device__ __forceinline__ int group_key0(const SlotLayout& sl, const int* s_blk, int bs, int g0, int gs) {
   if (!SPARSE) return gs;
   if (gs < sl.gen_start) {
-    const int i = gs / sl.pad_bs;
+    const int i = static_cast<int>(sl.pad_div.div(static_cast<uint32_t>(gs)));
     return s_blk[i] * bs + (gs - i * sl.pad_bs);
   }
   if (gs < sl.sink_start) return g0 + (gs - sl.gen_start);
@@ -115,7 +117,7 @@ template <bool SPARSE>
 __device__ __forceinline__ bool slot_valid(const SlotLayout& sl, int L, int bs, int G, int slot) {
   if (!SPARSE) return slot < L;
   if (slot < sl.gen_start) {
-    const int i = slot / sl.pad_bs;
+    const int i = static_cast<int>(sl.pad_div.div(static_cast<uint32_t>(slot)));
     const int r = slot - i * sl.pad_bs;
     return r < ((i == sl.nvb - 1) ? sl.last_size : bs);
   }
