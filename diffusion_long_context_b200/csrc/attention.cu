@@ -64,6 +64,7 @@ struct AttnArgs {
   int n_splits, tiles_per_split;
   int box_rows;           // rows per TMA box (divides 128)
   int gen_pad;            // slots of the current block in the sparse layout (multiple of box_rows)
+  FastDiv pad_div, bs_div;  // by round_up(bs, 8) and bs (host-computed)
   int S, C, bs, P, g0, g1;
   float scale_log2;
   int* dev_err;
@@ -147,10 +148,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (SPARSE) {
-    if (warp == 0)
-      build_sparse_layout(a.blocks + static_cast<size_t>(bh) * a.C, a.C,
-                          a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs, a.g0,
-                          a.g1, a.gen_pad, bk->blk, kMaxBlocks, bk->fsinks, kMaxSinks, &bk->sl);
+    if (warp == 0) {
+      const int32_t* blk_g = a.blocks + static_cast<size_t>(bh) * a.C;
+      const int32_t* snk_g = a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr;
+      build_sparse_layout(layout_prefetch(blk_g, a.C, snk_g, a.S), blk_g, a.C, snk_g, a.S, a.L, a.P, a.bs, a.g0, a.g1,
+                          a.gen_pad, a.box_rows, a.pad_div, a.bs_div, bk->blk, kMaxBlocks, bk->fsinks, kMaxSinks,
+                          &bk->sl);
+    }
   } else if (threadIdx.x == 0) {
     bk->sl.n_slots = a.L;
   }
@@ -734,7 +738,8 @@ int box_rows_for(bool sparse, int L, int bs, int G) {
   return pow2_rows((bs + 7) & ~7, cap);
 }
 
-// The current block is padded to whole boxes so that every box stays in one segment.
+// The sink segment and the current block are padded to whole boxes so that every box
+// stays in one segment.
 int gen_pad_for(int box_rows, int G) { return (G + box_rows - 1) / box_rows * box_rows; }
 
 
@@ -870,6 +875,13 @@ int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, 
   }
   args.box_rows = box_rows_for(SPARSE, args.L, args.bs, args.g1 - args.g0);
   args.gen_pad = gen_pad_for(args.box_rows, args.g1 - args.g0);
+  if (SPARSE) {
+    const int pad_bs = (args.bs + 7) & ~7;
+    const long long n_max = static_cast<long long>(args.C) * pad_bs + args.gen_pad +
+                            gen_pad_for(args.box_rows, std::min(args.S, kMaxSinks)) + 2 * kBN;
+    args.pad_div.init(static_cast<uint32_t>(pad_bs), static_cast<uint32_t>(std::min<long long>(n_max, 0xFFFFFFFFll)));
+    args.bs_div.init(static_cast<uint32_t>(std::max(args.bs, 1)), static_cast<uint32_t>(args.L));
+  }
   CUtensorMap mk, mv;
   int st = make_kv_map(&mk, args.K, args.B * args.Hkv, args.L, D, args.box_rows);
   if (st != FOCUS_OK) return st;
@@ -958,8 +970,9 @@ extern "C" size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, in
                                                int P, int g0, int g1) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || acap <= 0 || Hq % Hkv || bs <= 0 || C <= 0 || S < 0) return 0;
   const int nb = (P + bs - 1) / bs;
-  const long kv_cap = static_cast<long>(std::min(C, std::max(nb, 0))) * ((bs + 7) & ~7) +
-                      gen_pad_for(box_rows_for(true, L, bs, g1 - g0), g1 - g0) + std::min(S, kMaxSinks);
+  const int br = box_rows_for(true, L, bs, g1 - g0);
+  const long kv_cap = static_cast<long>(std::min(C, std::max(nb, 0))) * ((bs + 7) & ~7) + gen_pad_for(br, g1 - g0) +
+                      gen_pad_for(br, std::min(S, kMaxSinks));
   return plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(std::min<long>(kv_cap, 1 << 30)), false, L, S, C)
       .total;
 }
@@ -988,8 +1001,9 @@ extern "C" int focus_sparse_attention(const focus_bf16* Q_active, const int32_t*
   }
   if (B == 0) return FOCUS_OK;
   const int nb = (P + bs - 1) / bs;
-  const long kv_cap = static_cast<long>(std::min(C, nb)) * ((bs + 7) & ~7) +
-                      gen_pad_for(box_rows_for(true, L, bs, g1 - g0), g1 - g0) + S;
+  const int br = box_rows_for(true, L, bs, g1 - g0);
+  const long kv_cap = static_cast<long>(std::min(C, nb)) * ((bs + 7) & ~7) + gen_pad_for(br, g1 - g0) +
+                      gen_pad_for(br, S);
   FOCUS_CHECK_ARG(kv_cap < (1L << 30), "key set too large");
   const AttnPlan plan = plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(kv_cap), false, L, S, C);
   FOCUS_CHECK_ARG(ws_bytes >= plan.total && (plan.total == 0 || ws), "workspace too small: need %zu bytes, got %zu",

@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   const int dim = threadIdx.x % D, part = threadIdx.x / D;
   float acc = 0.f;
   const int rows = g * A;
+  FastDiv adiv;                                           // row r <-> (head r / A, row r % A)
+  adiv.init(static_cast<uint32_t>(max(A, 1)), static_cast<uint32_t>(rows + PARTS * 8));
   for (int r0 = part; r0 < rows; r0 += PARTS * 8) {       // 8 rows in flight per thread
     __nv_bfloat16 v[8];
 #pragma unroll
@@ -81,7 +83,8 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
       const int r = r0 + PARTS * u;
       v[u] = __float2bfloat16_rn(0.f);
       if (r < rows) {
-        const int hq = h * g + r / A, i = r % A;
+        const int rh = static_cast<int>(adiv.div(static_cast<uint32_t>(r)));
+        const int hq = h * g + rh, i = r - rh * A;
         v[u] = Q[((static_cast<size_t>(b) * Hq + hq) * acap + i) * D + dim];
       }
     }

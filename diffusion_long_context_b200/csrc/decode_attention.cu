@@ -61,6 +61,7 @@ struct DecArgs {
   int gen_pad;                 // slots of the current block (multiple of box_rows)
   int S, C, bs, P, g0, g1;
   float scale_log2;
+  FastDiv pad_div, bs_div, qcap_div;   // by round_up(bs, 8), bs and qcap (host-computed)
   int* dev_err;
 };
 
@@ -132,8 +133,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int nq_b = a.n_q ? min(a.n_q[b], a.qcap) : a.qcap;
   const int n_rows = a.g * a.qcap;             // <= NQ
   const int G = a.g1 - a.g0;
-  FastDiv qdiv;                                // query column q <-> (head q / qcap, row q % qcap)
-  qdiv.init(static_cast<uint32_t>(a.qcap), 64u);
+  const FastDiv qdiv = a.qcap_div;             // query column q <-> (head q / qcap, row q % qcap)
 
   // ---------------------------------------------------------------- prologue
   // The producer warp initialises the barriers, builds the slot layout and issues the first
@@ -146,11 +146,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const __nv_bfloat16* Vbh = a.V + static_cast<size_t>(bh) * a.L * D;
   int issued = 0;
   const uint64_t l2_stream = l2_evict_first_policy();   // K/V rows are read once per call
+  // kept-block list and sinks of this (b, h): their first entries are fetched right away
+  const int32_t* blk_g = FUSED ? bk->blk : a.blocks + static_cast<size_t>(bh) * a.C;
+  const int32_t* snk_g = a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr;
+  LayoutPrefetch pf{};
+  if (SPARSE && !FUSED && warp == kDecProducerWarp) pf = layout_prefetch(blk_g, a.C, snk_g, a.S);
   SlotLayout sl_p{};
   int p_n = 0;                 // tiles of this (b, h)
   bool p_more = true;          // the end marker is not issued yet
-  // fetch tile `tile` into ring stage `it % STAGES`: TMA boxes from parallel lanes
-  auto produce = [&](int it, int tile) {
+  // fetch tile `tile` into ring stage `it % STAGES`: TMA boxes from parallel lanes, rows
+  // outside key runs by cp.async. With `defer`, a stage that used cp.async is left
+  // un-arrived (returns true): the caller completes it with finish_deferred.
+  auto produce = [&](int it, int tile, bool defer) -> bool {
     const int s = it % STAGES;
     const int slot0 = tile * 128;
     uint8_t* dK = sK + s * SM::kTile;
@@ -184,6 +191,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           cp_async16(smem_u32(dV + sw128_offset(row, c, 128)), Vbh + koff, src_bytes);
         }
       }
+      if (defer) {
+        if (lane == 0) bk->stage_tile[s] = tile;
+        __syncwarp();
+        ++issued;
+        return true;
+      }
       cp_async_wait_all();
       fence_proxy_async_smem();
     }
@@ -194,6 +207,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     __syncwarp();
     ++issued;
+    return false;
+  };
+  // complete the deferred stages (bit s of `stages`) once their cp.async rows have landed
+  auto finish_deferred = [&](unsigned stages) {
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0)
+      for (int st = 0; st < STAGES; ++st)
+        if ((stages >> st) & 1u) mbar_arrive(&bk->full[st]);
+    __syncwarp();
   };
   // no more tiles: stage `it % STAGES` carries the end marker (plain arrive, no bytes)
   auto produce_end = [&](int it) {
@@ -233,6 +257,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     {
       // qbar: 3 row groups x 64 dim pairs; 8 rows in flight per thread
       const int t = threadIdx.x, dp = t % 64, rg = t / 64;
+      FastDiv rdiv;                                            // row r <-> (head r / nq_b, row r % nq_b)
+      rdiv.init(static_cast<uint32_t>(max(nq_b, 1)), static_cast<uint32_t>(rows + 64));
       float2 acc = make_float2(0.f, 0.f);
       for (int r0 = rg; r0 < rows; r0 += 3 * 8) {
         __nv_bfloat162 v[8];
@@ -241,7 +267,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           const int r = r0 + 3 * u;
           v[u] = __floats2bfloat162_rn(0.f, 0.f);
           if (r < rows) {
-            const int hq = kvh * a.g + r / nq_b, i = r % nq_b;
+            const int rh = static_cast<int>(rdiv.div(static_cast<uint32_t>(r)));
+            const int hq = kvh * a.g + rh, i = r - rh * nq_b;
             v[u] = *reinterpret_cast<const __nv_bfloat162*>(
                 a.Q + ((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D + 2 * dp);
           }
@@ -311,15 +338,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tma_prefetch_desc(&tmV);
     }
     if (SPARSE) {
-      sl_p = build_sparse_layout(FUSED ? bk->blk : a.blocks + static_cast<size_t>(bh) * a.C, a.C,
-                                 a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr, a.S, a.L, a.P, a.bs,
-                                 a.g0, a.g1, a.gen_pad, bk->blk, kDecMaxBlocks, bk->sinks, kDecMaxSinks, &bk->sl);
+      if (FUSED) pf = layout_prefetch(blk_g, a.C, snk_g, a.S);
+      sl_p = build_sparse_layout(pf, blk_g, a.C, snk_g, a.S, a.L, a.P, a.bs, a.g0, a.g1, a.gen_pad, a.box_rows,
+                                 a.pad_div, a.bs_div, bk->blk, kDecMaxBlocks, bk->sinks, kDecMaxSinks, &bk->sl);
     } else {
       sl_p.n_slots = a.L;
       if (lane == 0) bk->sl = sl_p;
     }
     p_n = (sl_p.n_slots + 127) / 128;
     __syncwarp();
+    // the layout and the barriers are ready: release the other warps, then fill the ring
+    // (a tile gathered row by row completes after the TMA tiles behind it are issued)
+    named_bar_arrive(2, kDecThreads);
+    unsigned deferred = 0;
     for (int it = 0; it < STAGES; ++it) {
       const int tile = rank + it * cs;
       if (tile >= p_n) {
@@ -327,8 +358,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         p_more = false;
         break;
       }
-      produce(it, tile);
+      if (produce(it, tile, true)) deferred |= 1u << it;
     }
+    if (deferred) finish_deferred(deferred);
+    if (!FUSED && cs > 1) cluster_wait();   // the claim counter is initialised
   }
   if (warp == kDecMmaWarp) {
     tmem_alloc(&bk->tmem_base, SM::kTmemCols);
@@ -361,10 +394,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     fence_proxy_async_smem();
   }
-  tc_fence_before();
-  if (!FUSED && cs > 1) cluster_wait();
-  __syncthreads();
-  tc_fence_after();
+  if (warp != kDecProducerWarp) {
+    tc_fence_before();
+    named_bar_sync(2, kDecThreads);      // layout, barriers, TMEM and Q are ready
+    tc_fence_after();
+    if (!FUSED && cs > 1) cluster_wait();
+  }
 
   const uint32_t tmem = bk->tmem_base;
   const SlotLayout sl = bk->sl;
@@ -396,7 +431,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int tile = next;
         if (lane == 0) next = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));   // claim ahead
         next = __shfl_sync(0xffffffffu, next, 0);
-        produce(it, tile);
+        produce(it, tile, false);
       }
     }
     // wait for the copies still in flight; the end marker (issue index `issued`) shares its
@@ -433,10 +468,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int s = it % STAGES, sb = it & 1;
         if (!mbar_wait(&bk->full[s], (it / STAGES) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
         if (bk->stage_tile[s] < 0) {
-          // end marker: finish the last tile, then release the softmax warps
-          if (it > 0) ok = issue_pv(it - 1);
+          // end marker: release the softmax warps (they wait for the last PV's completion
+          // on pv_done), then finish the last tile
           n_it = it;
           mbar_arrive(&bk->s_full[sb]);
+          if (it > 0) ok = issue_pv(it - 1);
           break;
         }
         if (it >= 2 && !mbar_wait(&bk->s_free[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
@@ -840,6 +876,14 @@ int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bflo
   } else {
     a.box_rows = cap;
     a.gen_pad = 0;
+  }
+  {
+    const int pad_bs = (bs + 7) & ~7;
+    const long long n_max = static_cast<long long>(C) * pad_bs + a.gen_pad +
+                            (std::min(S, kDecMaxSinks) + a.box_rows - 1) / a.box_rows * a.box_rows + 256;
+    a.pad_div.init(static_cast<uint32_t>(pad_bs), static_cast<uint32_t>(std::min<long long>(n_max, 0xFFFFFFFFll)));
+    a.bs_div.init(static_cast<uint32_t>(std::max(bs, 1)), static_cast<uint32_t>(L));
+    a.qcap_div.init(static_cast<uint32_t>(qcap), 64u);
   }
   const int nrows = a.g * qcap;
   if (kbar) {

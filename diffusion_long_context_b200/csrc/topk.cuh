@@ -2,8 +2,9 @@
 //
 // Order: larger key first, ties to the lower index. Keys are order-preserving 32-bit
 // images of the scores (float_order_key), so -0.0 and +0.0 tie.
-//   1. Radix select, 8 bits per pass (4 passes), finds T = the k-th largest key and how
-//      many keys equal to T are taken. Histograms use warp-aggregated shared atomics
+//   1. Radix select, 8 bits per pass (at most 4 passes), finds T = the k-th largest key
+//      and how many keys equal to T are taken. A pass whose boundary digit is taken
+//      whole ends the search early: T is then a prefix, compared under its mask. Histograms use warp-aggregated shared atomics
 //      (lanes with the same digit add once), so a digit shared by every key does not
 //      serialise the CTA; one warp locates the digit with a lane-parallel suffix scan.
 //   2. Ordered selection: each warp owns a contiguous segment of indices; a first walk
@@ -40,6 +41,7 @@ struct TopkShared {
   int w_gt[32];
   int w_eq[32];
   uint32_t prefix;
+  uint32_t mask;           // bits of prefix that are fixed
   int remaining;
 };
 
@@ -60,6 +62,7 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
   }
   if (tid == 0) {
     sm.prefix = 0u;
+    sm.mask = 0u;
     sm.remaining = k;
   }
   for (int pass = 0; pass < 4; ++pass) {
@@ -100,22 +103,28 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
       if (lane == L) {
         int cum = incl - own;
         int digit = 0;
+        int whole = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (cum + c[j] >= rem) {
             digit = 255 - 8 * lane - j;
+            whole = c[j];
             break;
           }
           cum += c[j];
         }
         sm.remaining = rem - cum;
         sm.prefix = prefix | (static_cast<uint32_t>(digit) << shift);
+        // the digit's keys are all taken: no lower bit can change the selection
+        sm.mask = (whole == rem - cum) ? (0xFFFFFFFFu << shift) : 0u;
       }
     }
     __syncthreads();
+    if (sm.mask != 0u) break;
   }
   const uint32_t T = sm.prefix;
-  const int take_eq = sm.remaining;              // keys equal to T to keep (lowest indices first)
+  const uint32_t M = sm.mask != 0u ? sm.mask : 0xFFFFFFFFu;   // a full search fixes every bit
+  const int take_eq = sm.remaining;              // keys equal to T (under M) to keep, lowest indices first
   // ordered selection over warp-owned contiguous segments
   const int seg = ((n + nwarps - 1) / nwarps + 31) & ~31;
   const int w_begin = min(n, warp * seg), w_end = min(n, w_begin + seg);
@@ -123,7 +132,7 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
   for (int base = w_begin; base < w_end; base += 32) {
     const int i = base + lane;
     uint32_t key = 0u;
-    if (i < w_end) key = key_of(i);
+    if (i < w_end) key = key_of(i) & M;
     gt += __popc(__ballot_sync(0xffffffffu, i < w_end && key > T));
     eq += __popc(__ballot_sync(0xffffffffu, i < w_end && key == T));
   }
@@ -143,7 +152,7 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
   for (int base = w_begin; base < w_end; base += 32) {
     const int i = base + lane;
     uint32_t key = 0u;
-    if (i < w_end) key = key_of(i);
+    if (i < w_end) key = key_of(i) & M;
     const bool is_gt = i < w_end && key > T;
     const bool is_eq = i < w_end && key == T;
     const unsigned meq = __ballot_sync(0xffffffffu, is_eq);
