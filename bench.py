@@ -31,6 +31,10 @@ sys.path.insert(0, ROOT)
 
 from diffusion_long_context_b200 import configs, inputs  # noqa: E402
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one sparse-attention launch
+# on this workload, from the committed ncu summary of the sparse decode kernel. It is reset
+# to None whenever that kernel changes, until it is captured again.
+SPARSE_TRAFFIC_BYTES = 69.82e6
 METRIC = "sparse dLLM attn step latency & active tok/s at 32K ctx; % of HBM/TC roofline"
 CFG = configs.FULL_32K
 
@@ -429,7 +433,7 @@ def run_ours(args):
                        "l2": "inputs larger than L2: 17.2 GB of K/V per step, every layer distinct",
                        "replay": "one CUDA graph per step", "parallelism": f"replicas x{ws}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": None,
+                         "frac": achieved / hbm, "traffic": SPARSE_TRAFFIC_BYTES,
                          "kernel": "focus_sparse_attention (decode kernel, cluster split), one layer; CUDA-graph "
                                    "replay of all sparse layers",
                          "bytes_per_launch": sparse_bytes, "flops_per_launch": sparse_flops,

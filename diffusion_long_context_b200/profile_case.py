@@ -1,6 +1,6 @@
 """One-layer workload for kernel profiling (ncu) of a single Focus-dLLM call.
 
-  python -m diffusion_long_context_b200.profile_case --call sparse|dense|colsum|select|blocks|means|refresh \
+  python -m diffusion_long_context_b200.profile_case --call sparse|fused|dense|colsum|select|blocks|means|refresh \
       [--L 32768] [--repeat 3]
 
 Builds one layer of the 32K LLaDA-shaped step (synthetic, seeded), runs the whole step
@@ -21,7 +21,7 @@ from . import focus as F
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--call", default="sparse",
-                    choices=["sparse", "dense", "colsum", "select", "blocks", "means", "refresh"])
+                    choices=["sparse", "fused", "dense", "colsum", "select", "blocks", "means", "refresh"])
     ap.add_argument("--L", type=int, default=32768)
     ap.add_argument("--repeat", type=int, default=3)
     a = ap.parse_args()
@@ -66,6 +66,10 @@ def main():
     def sparse():
         F.focus_sparse_attention(Qa, n_active, K, V, sinks, blocks, c.bs, c.P, c.g0, c.g1, O, ws=ws)
 
+    def fused():
+        F.focus_sparse_attention_fused(Qa, n_active, K, V, kbar, c.C, sinks, c.bs, c.P, c.g0, c.g1, blocks, O,
+                                       ws=ws)
+
     O_full = None
 
     def refresh():
@@ -79,7 +83,7 @@ def main():
     torch.cuda.synchronize()
     if a.call == "refresh":
         O_full = torch.empty((c.B, c.Hq, c.L, c.d), dtype=torch.bfloat16, device=dev)
-    fn = {"sparse": sparse, "dense": dense, "colsum": dense_colsum, "select": select, "blocks": blocks_sel,
+    fn = {"sparse": sparse, "fused": fused, "dense": dense, "colsum": dense_colsum, "select": select, "blocks": blocks_sel,
           "means": means, "refresh": refresh}[a.call]
     for _ in range(a.repeat):
         fn()
