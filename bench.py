@@ -31,10 +31,11 @@ sys.path.insert(0, ROOT)
 
 from diffusion_long_context_b200 import configs, inputs  # noqa: E402
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one sparse-attention launch
-# on this workload, from the committed ncu summary of the sparse decode kernel. It is reset
-# to None whenever that kernel changes, until it is captured again.
-SPARSE_TRAFFIC_BYTES = 69.82e6
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the step's
+# dominant kernel on this workload, from the committed ncu summaries: the fused sparse
+# layer (default step) and the unfused sparse attention. Each is reset to None whenever
+# its kernel changes, until it is captured again.
+TRAFFIC_BYTES = {"fused": None, "sparse": None}
 METRIC = "sparse dLLM attn step latency & active tok/s at 32K ctx; % of HBM/TC roofline"
 CFG = configs.FULL_32K
 
@@ -256,7 +257,7 @@ def run_ours(args):
     from diffusion_long_context_b200.step import SparseStep
 
     cfg, st, Q_full, K, V = build_replica(CFG, dev, seed_offset=rank)
-    step = SparseStep(cfg, Q_full, K, V, device=dev)
+    step = SparseStep(cfg, Q_full, K, V, device=dev, fused=not args.unfused)
     step.set_state(torch.from_numpy(st.conf_prev), torch.from_numpy(st.mask), non_blocking=False)
 
     # ---- block entry: block means of the 29 sparse layers (timed once, after a warm run)
@@ -350,10 +351,20 @@ def run_ours(args):
     sparse_flops = 4.0 * A * g * mean_ip * c.d
     dense_bytes = c.B * c.Hkv * c.L * c.d * 2 * 2 + 2 * c.B * c.Hq * A * c.d * 2
     kbar_bytes = c.B * c.Hkv * c.nb * c.d * 4
-    # the step runs focus_block_select then focus_sparse_attention per sparse layer; the
-    # roofline reports the attention launch (gathered K/V + Q + O bytes)
-    t_sp = call_ms["sparse_attention"] * 1e-3
-    achieved = sparse_bytes / t_sp / 1e9
+    # the step runs one fused launch per sparse layer (kbar + gathered K/V + Q + O + the
+    # kept-block list), or focus_block_select then focus_sparse_attention (the attention
+    # launch is reported: gathered K/V + Q + O)
+    blocks_bytes = c.B * c.Hkv * c.C * 4
+    if step.fused:
+        dom_kind, dom_bytes, dom_call = "fused", sparse_bytes + kbar_bytes + blocks_bytes, "sparse_layer_fused"
+        dom_name = ("focus_sparse_attention_fused (decode kernel with the relevance/top-C prologue, cluster "
+                    "split), one layer; CUDA-graph replay of all sparse layers")
+    else:
+        dom_kind, dom_bytes, dom_call = "sparse", sparse_bytes, "sparse_attention"
+        dom_name = ("focus_sparse_attention (decode kernel, cluster split), one layer; CUDA-graph replay of all "
+                    "sparse layers")
+    t_sp = call_ms[dom_call] * 1e-3
+    achieved = dom_bytes / t_sp / 1e9
     # step roofline: slower of bytes at HBM peak and flops at the tensor peak, summed over calls
     n_dense, n_sparse = c.l_dense + 1, c.n_layers - c.l_dense - 1
     colsum_bytes = c.B * c.Hkv * c.L * c.d * 2
@@ -431,13 +442,13 @@ def run_ours(args):
                        "d": c.d, "layers": c.n_layers, "l_dense": c.l_dense, "n_t": c.n_t, "rho": c.rho,
                        "w": c.w, "bs": c.bs, "C": c.C, "S": c.S, "n_active": n_act,
                        "l2": "inputs larger than L2: 17.2 GB of K/V per step, every layer distinct",
-                       "replay": "one CUDA graph per step", "parallelism": f"replicas x{ws}"},
+                       "replay": "one CUDA graph per step",
+                       "sparse_layer": "fused relevance/top-C + attention" if step.fused else "two calls",
+                       "parallelism": f"replicas x{ws}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": SPARSE_TRAFFIC_BYTES,
-                         "kernel": "focus_sparse_attention (decode kernel, cluster split), one layer; CUDA-graph "
-                                   "replay of all sparse layers",
-                         "bytes_per_launch": sparse_bytes, "flops_per_launch": sparse_flops,
-                         "launch_ms": call_ms["sparse_attention"], "peak_source": f"{peak_kind} hbm_gbs"},
+                         "frac": achieved / hbm, "traffic": TRAFFIC_BYTES[dom_kind],
+                         "kernel": dom_name, "bytes_per_launch": dom_bytes, "flops_per_launch": sparse_flops,
+                         "launch_ms": call_ms[dom_call], "peak_source": f"{peak_kind} hbm_gbs"},
             "step_roofline": {"bytes": step_bytes, "roofline_ms": step_roof_ms, "frac": step_roof_ms / ms_step},
             "calls_ms": call_ms,
             "dense_comparator": {"ms": dense_cmp_ms, "kept_kv_ratio": kept_ratio,
@@ -469,6 +480,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--skip-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--skip-refresh", action="store_true", help="skip the full-refresh comparator")
+    ap.add_argument("--unfused", action="store_true",
+                    help="run block select and sparse attention as two launches per sparse layer")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

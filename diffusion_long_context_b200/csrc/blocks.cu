@@ -58,7 +58,7 @@ constexpr int kSelectThreads = 512;
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
     const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ n_active, const float* __restrict__ kbar, int Hq,
-    int Hkv, int acap, int nb, int C, int32_t* __restrict__ blocks, float* __restrict__ scores) {
+    int Hkv, int acap, FastDiv acap_div, int nb, int C, int32_t* __restrict__ blocks, float* __restrict__ scores) {
   griddep_wait();               // inputs may come from the previous kernel on the stream
   griddep_launch_dependents();
   constexpr int PARTS = kSelectThreads / D;
@@ -74,22 +74,25 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   const int dim = threadIdx.x % D, part = threadIdx.x / D;
   float acc = 0.f;
   const int rows = g * A;
-  FastDiv adiv;                                           // row r <-> (head r / A, row r % A)
-  adiv.init(static_cast<uint32_t>(max(A, 1)), static_cast<uint32_t>(rows + PARTS * 8));
-  for (int r0 = part; r0 < rows; r0 += PARTS * 8) {       // 8 rows in flight per thread
+  // Row slot r = (head r / acap, position r % acap). Every slot is loaded and positions
+  // >= A are masked afterwards, so the loads do not wait for n_active.
+  const int nr = g * acap;
+  for (int r0 = part; r0 < nr; r0 += PARTS * 8) {         // 8 rows in flight per thread
     __nv_bfloat16 v[8];
+    int pos[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int r = r0 + PARTS * u;
       v[u] = __float2bfloat16_rn(0.f);
-      if (r < rows) {
-        const int rh = static_cast<int>(adiv.div(static_cast<uint32_t>(r)));
-        const int hq = h * g + rh, i = r - rh * A;
-        v[u] = Q[((static_cast<size_t>(b) * Hq + hq) * acap + i) * D + dim];
+      pos[u] = acap;
+      if (r < nr) {
+        const int rh = static_cast<int>(acap_div.div(static_cast<uint32_t>(r)));
+        pos[u] = r - rh * acap;
+        v[u] = Q[((static_cast<size_t>(b) * Hq + h * g + rh) * acap + pos[u]) * D + dim];
       }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) acc += __bfloat162float(v[u]);
+    for (int u = 0; u < 8; ++u) acc += pos[u] < A ? __bfloat162float(v[u]) : 0.f;
   }
   s_part[part][dim] = acc;
   __syncthreads();
@@ -140,8 +143,12 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   if (cs > 1) cluster_sync();   // every share of R is in CTA 0
   else __syncthreads();
   if (rank != 0) return;
-  block_topk_ascending([&](int i) { return float_order_key(s_R[i]); }, nb, C, blocks + static_cast<size_t>(bh) * C, C,
-                       tk);
+  int32_t* out = blocks + static_cast<size_t>(bh) * C;
+  auto key_of = [&](int i) { return float_order_key(s_R[i]); };
+  if (nb <= kSelectThreads) block_topk_small<1>(key_of, nb, C, out, C, tk);
+  else if (nb <= 2 * kSelectThreads) block_topk_small<2>(key_of, nb, C, out, C, tk);
+  else if (nb <= 4 * kSelectThreads) block_topk_small<4>(key_of, nb, C, out, C, tk);
+  else block_topk_ascending(key_of, nb, C, out, C, tk);
 }
 
 }  // namespace focus
@@ -194,6 +201,8 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(Q_active);
   // cluster of cs CTAs per (sequence, KV head), cs a power of two with B*Hkv*cs <= SMs
+  FastDiv acap_div;
+  acap_div.init(static_cast<uint32_t>(acap), static_cast<uint32_t>(Hq / Hkv) * static_cast<uint32_t>(acap) + 4096u);
   const int units = B * Hkv;
   int cs = 1;
   while (cs < 8 && units * cs * 2 <= device_sm_count() && (nb + cs * 2 - 1) / (cs * 2) >= 16) cs *= 2;
@@ -205,7 +214,7 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
       cfg = true;
     }
     err = launch_k_cluster(block_select_kernel<128>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
-                           n_active, kbar, Hq, Hkv, acap, nb, C, blocks, scores_opt);
+                           n_active, kbar, Hq, Hkv, acap, acap_div, nb, C, blocks, scores_opt);
   } else {
     static bool cfg = false;
     if (!cfg) {
@@ -213,7 +222,7 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
       cfg = true;
     }
     err = launch_k_cluster(block_select_kernel<64>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
-                           n_active, kbar, Hq, Hkv, acap, nb, C, blocks, scores_opt);
+                           n_active, kbar, Hq, Hkv, acap, acap_div, nb, C, blocks, scores_opt);
   }
   note_launch();
   if (err != cudaSuccess) {

@@ -246,7 +246,36 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int j_begin = rank * chunk, j_end = min(a.nb, j_begin + chunk);
     uint32_t* s_key = reinterpret_cast<uint32_t*>(s_R);
     const uint32_t sK0 = smem_u32(s_key);
-    // this thread's first kbar row is fetched before qbar is known (the two loads overlap)
+    // qbar over the group's active rows: 3 row groups x 64 dim pairs, 8 rows in flight per
+    // thread. Row slot r = (head r / qcap, position r % qcap); every slot is loaded and the
+    // positions >= nq_b are masked afterwards, so the loads do not wait for n_q. The first
+    // batch of Q rows is requested before this thread's first kbar row, so the
+    // latency-critical Q loads are not queued behind it.
+    const int t = threadIdx.x, dp = t % 64, rg = t / 64;
+    const int nr = a.g * a.qcap;
+    auto load8 = [&](int r0, __nv_bfloat162 (&v)[8]) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = r0 + 3 * u;
+        v[u] = __floats2bfloat162_rn(0.f, 0.f);
+        if (r < nr) {
+          const int rh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
+          const int i = r - rh * a.qcap;
+          v[u] = *reinterpret_cast<const __nv_bfloat162*>(
+              a.Q + ((static_cast<size_t>(b) * a.Hq + kvh * a.g + rh) * a.qcap + i) * D + 2 * dp);
+        }
+      }
+    };
+    auto mask8 = [&](int r0, __nv_bfloat162 (&v)[8]) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int r = r0 + 3 * u;
+        const int rh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
+        if (r - rh * a.qcap >= nq_b) v[u] = __floats2bfloat162_rn(0.f, 0.f);
+      }
+    };
+    __nv_bfloat162 qv8[8];
+    load8(rg, qv8);
     int j = j_begin + threadIdx.x;
     float4 kv[D / 4];
     if (j < j_end) {
@@ -255,30 +284,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       for (int c = 0; c < D / 4; ++c) kv[c] = __ldg(row + c);
     }
     {
-      // qbar: 3 row groups x 64 dim pairs; 8 rows in flight per thread
-      const int t = threadIdx.x, dp = t % 64, rg = t / 64;
-      FastDiv rdiv;                                            // row r <-> (head r / nq_b, row r % nq_b)
-      rdiv.init(static_cast<uint32_t>(max(nq_b, 1)), static_cast<uint32_t>(rows + 64));
       float2 acc = make_float2(0.f, 0.f);
-      for (int r0 = rg; r0 < rows; r0 += 3 * 8) {
-        __nv_bfloat162 v[8];
+      for (int r0 = rg;;) {
+        mask8(r0, qv8);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int r = r0 + 3 * u;
-          v[u] = __floats2bfloat162_rn(0.f, 0.f);
-          if (r < rows) {
-            const int rh = static_cast<int>(rdiv.div(static_cast<uint32_t>(r)));
-            const int hq = kvh * a.g + rh, i = r - rh * nq_b;
-            v[u] = *reinterpret_cast<const __nv_bfloat162*>(
-                a.Q + ((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D + 2 * dp);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float2 f = __bfloat1622float2(v[u]);
+          const float2 f = __bfloat1622float2(qv8[u]);
           acc.x += f.x;
           acc.y += f.y;
         }
+        r0 += 3 * 8;
+        if (r0 >= nr) break;
+        load8(r0, qv8);
       }
       s_part[rg * D + 2 * dp] = acc.x;
       s_part[rg * D + 2 * dp + 1] = acc.y;
@@ -314,7 +331,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     if (cs > 1) cluster_sync();   // every CTA holds all nb keys
     else __syncthreads();
-    block_topk_ascending([&](int i) { return s_key[i]; }, a.nb, a.C, bk->blk, a.C, bk->tk);
+    auto key_of = [&](int i) { return s_key[i]; };
+    if (a.nb <= 4 * kDecThreads) block_topk_small<4>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
+    else if (a.nb <= 8 * kDecThreads) block_topk_small<8>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
+    else block_topk_ascending(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
     __syncthreads();
     if (rank == 0 && a.blocks_out)
       for (int i = threadIdx.x; i < a.C; i += kDecThreads) a.blocks_out[static_cast<size_t>(bh) * a.C + i] = bk->blk[i];

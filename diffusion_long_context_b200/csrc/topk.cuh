@@ -1,15 +1,19 @@
 // Block-wide top-k selection shared by the block (top-C) and sink (top-S) kernels.
 //
 // Order: larger key first, ties to the lower index. Keys are order-preserving 32-bit
-// images of the scores (float_order_key), so -0.0 and +0.0 tie.
-//   1. Radix select, 8 bits per pass (at most 4 passes), finds T = the k-th largest key
-//      and how many keys equal to T are taken. A pass whose boundary digit is taken
-//      whole ends the search early: T is then a prefix, compared under its mask. Histograms use warp-aggregated shared atomics
-//      (lanes with the same digit add once), so a digit shared by every key does not
-//      serialise the CTA; one warp locates the digit with a lane-parallel suffix scan.
-//   2. Ordered selection: each warp owns a contiguous segment of indices; a first walk
-//      counts keys > T and == T per warp, one block barrier turns the counts into
-//      offsets, and a second walk writes the selected indices in ascending order.
+// images of the scores (float_order_key), so -0.0 and +0.0 tie. Two forms:
+//   block_topk_small (n <= KPT * blockDim.x): keys in registers, offset by the block
+//     minimum; the first 8-bit radix digit is the top of the spanned range, so smooth
+//     scores spread over the 256 bins and one or two passes usually fix the k-th key.
+//     One packed (greater, equal) block scan then places the selection in index order.
+//   block_topk_ascending (any n): keys read through key_of each pass.
+//     1. Radix select, 8 bits per pass (at most 4 passes), finds T = the k-th largest key
+//        and how many keys equal to T are taken. Histograms use warp-aggregated shared
+//        atomics; one warp locates the digit with a lane-parallel suffix scan. A pass
+//        whose boundary digit is taken whole ends the search early.
+//     2. Ordered selection: each warp owns a contiguous segment of indices; a first walk
+//        counts keys > T and == T per warp, one block barrier turns the counts into
+//        offsets, and a second walk writes the selected indices in ascending order.
 #pragma once
 
 #include "focus_common.cuh"
@@ -37,6 +41,7 @@ __device__ __forceinline__ int block_excl_scan(bool flag, int* s_warp, int& tota
 
 struct TopkShared {
   int hist[256];
+  int hist2[256];          // second histogram (block_topk_small alternates the two)
   int s_warp[32];
   int w_gt[32];
   int w_eq[32];
@@ -164,6 +169,185 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
     run_sel += __popc(msel);
   }
   for (int i = k + tid; i < cap; i += nt) out[i] = -1;
+}
+
+// Top-k for small n (n <= KPT * blockDim.x): same contract and order as
+// block_topk_ascending. Thread t holds the keys of indices [KPT*t, KPT*t + KPT) in
+// registers. The keys are first offset by the block minimum, and the first radix digit is
+// the top 8 bits of the range actually spanned (max - min), so a smooth score
+// distribution spreads over all 256 bins and one or two passes usually find the k-th key.
+// The two histograms alternate, so each pass needs two block barriers. The ordered
+// output comes from one block scan of per-thread (greater, equal) counts packed in one
+// word (n < 65536).
+// key[j] holds the key of index KPT * threadIdx.x + j (any value when that index >= n).
+// key[j] holds the key of index KPT * threadIdx.x + j (any value when that index >= n);
+// the array is overwritten.
+// priv (optional): 2 * (blockDim.x / 32) * 257 ints of shared memory for per-warp
+// histograms (padded so that the warps' copies of a bin sit in different banks); with it
+// a bin holding most of the keys costs no cross-warp atomic serialisation.
+template <int KPT>
+__device__ void block_topk_small_regs(uint32_t (&key)[KPT], int n, int k, int32_t* out, int cap,
+                                      TopkShared& sm, int* priv = nullptr) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
+  k = min(k, n);
+  if (k <= 0) {
+    for (int i = tid; i < cap; i += nt) out[i] = -1;
+    return;
+  }
+  if (k >= n) {
+    for (int i = tid; i < cap; i += nt) out[i] = (i < n) ? i : -1;
+    return;
+  }
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if (tid * KPT + j < n) {
+      kmin = min(kmin, key[j]);
+      kmax = max(kmax, key[j]);
+    }
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    sm.w_gt[warp] = static_cast<int>(kmin);
+    sm.w_eq[warp] = static_cast<int>(kmax);
+  }
+  for (int i = tid; i < 256; i += nt) sm.hist[i] = 0;
+  if (priv)
+    for (int i = tid; i < nwarps * 257; i += nt) priv[i] = 0;
+  __syncthreads();
+  for (int w = 0; w < nwarps; ++w) {
+    kmin = min(kmin, static_cast<uint32_t>(sm.w_gt[w]));
+    kmax = max(kmax, static_cast<uint32_t>(sm.w_eq[w]));
+  }
+  // relative keys rk = key - kmin in [0, range] (in place); fixed part: rk >> hi == P
+  const uint32_t range = kmax - kmin;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) key[j] -= kmin;
+  int hi = 32 - __clz(range);          // bits spanned (0 when every key is equal)
+  uint32_t P = 0u;
+  int remaining = k;
+  int buf = 0;
+  bool whole = (range == 0u);          // all keys equal: take the lowest indices
+  while (hi > 0 && !whole) {
+    const int lo = max(0, hi - 8);
+    int* hist = buf ? sm.hist2 : sm.hist;
+    int* other = buf ? sm.hist : sm.hist2;
+    int* whist = hist;                   // where this warp counts
+    if (priv) {
+      int* pcur = priv + buf * nwarps * 257;
+      int* poth = priv + (buf ^ 1) * nwarps * 257;
+      for (int i = tid; i < nwarps * 257; i += nt) poth[i] = 0;   // cleared for the next pass
+      whist = pcur + warp * 257;
+    } else {
+      for (int i = tid; i < 256; i += nt) other[i] = 0;           // cleared for the next pass
+    }
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      const int i = tid * KPT + j;
+      const uint32_t rk = key[j];
+      if (i < n && (hi >= 32 || (rk >> hi) == P)) atomicAdd(&whist[(rk >> lo) & ((1u << (hi - lo)) - 1u)], 1);
+    }
+    __syncthreads();
+    if (priv) {
+      const int* pcur = priv + buf * nwarps * 257;
+      for (int b = tid; b < 256; b += nt) {
+        int tot = 0;
+        for (int w = 0; w < nwarps; ++w) tot += pcur[w * 257 + b];
+        hist[b] = tot;
+      }
+      __syncthreads();
+    }
+    // every warp locates the digit holding the remaining-th largest candidate (no extra
+    // barrier: each warp reaches the same answer from the same counts). Lane l owns
+    // digits 255-8l .. 248-8l in descending order.
+    {
+      int c[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) c[jj] = hist[255 - 8 * lane - jj];
+      int pre[8];
+      pre[0] = c[0];
+#pragma unroll
+      for (int jj = 1; jj < 8; ++jj) pre[jj] = pre[jj - 1] + c[jj];
+      const int own = pre[7];
+      int incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int excl = incl - own;
+      const unsigned hit = __ballot_sync(0xffffffffu, incl >= remaining);
+      const int L = __ffs(hit) - 1;
+      // in lane L: the first jj with excl + pre[jj] >= remaining (branch-free)
+      int jsel = 0;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) jsel += (excl + pre[jj] < remaining) ? 1 : 0;
+      int before = excl, cnt = 0;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        before += (jj < jsel) ? c[jj] : 0;
+        cnt = (jj == jsel) ? c[jj] : cnt;
+      }
+      const int digit = __shfl_sync(0xffffffffu, 255 - 8 * lane - jsel, L);
+      cnt = __shfl_sync(0xffffffffu, cnt, L);
+      remaining -= __shfl_sync(0xffffffffu, before, L);
+      whole = (cnt == remaining);
+      P = (P << (hi - lo)) | static_cast<uint32_t>(digit);
+      hi = lo;
+    }
+    buf ^= 1;
+    __syncthreads();                   // this pass's histogram is read before it is cleared again
+  }
+  // keys above the threshold: (rk >> hi) > P; at the threshold: == P (hi = 0 after a
+  // full search; every key when all are equal, P = 0)
+  const int take_eq = remaining;
+  int gt = 0, eq = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int i = tid * KPT + j;
+    const uint32_t v = (hi >= 32) ? 0u : (key[j] >> hi);
+    gt += (i < n && v > P) ? 1 : 0;
+    eq += (i < n && v == P) ? 1 : 0;
+  }
+  // exclusive block scan of (gt | eq << 16) in thread order == index order
+  const int packed = gt | (eq << 16);
+  int incl = packed;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) sm.s_warp[warp] = incl;
+  __syncthreads();
+  int before = incl - packed;
+  for (int w = 0; w < warp; ++w) before += sm.s_warp[w];
+  int gtb = before & 0xFFFF, eqb = before >> 16;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int i = tid * KPT + j;
+    const uint32_t v = (hi >= 32) ? 0u : (key[j] >> hi);
+    const bool is_gt = i < n && v > P;
+    const bool is_eq = i < n && v == P;
+    const bool sel = is_gt || (is_eq && eqb < take_eq);
+    const int pos = gtb + min(eqb, take_eq);
+    if (sel && pos < cap) out[pos] = i;
+    gtb += is_gt ? 1 : 0;
+    eqb += is_eq ? 1 : 0;
+  }
+  for (int i = k + tid; i < cap; i += nt) out[i] = -1;
+}
+
+template <int KPT, typename KeyFn>
+__device__ void block_topk_small(KeyFn key_of, int n, int k, int32_t* out, int cap, TopkShared& sm) {
+  uint32_t key[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int i = threadIdx.x * KPT + j;
+    key[j] = i < n ? key_of(i) : 0u;
+  }
+  block_topk_small_regs<KPT>(key, n, k, out, cap, sm);
 }
 
 }  // namespace focus

@@ -3,8 +3,8 @@
 A non-block-entry step (Focus-dLLM summary page, "方法步骤详情" / method steps (1)-(5)):
   select_queries -> gather the active query rows of every layer -> layers 0..l_dense:
   dense attention (layer l_dense also produces the sink column sums) -> sink top-S ->
-  layers > l_dense: block relevance + top-C, then sparse attention over sinks U blocks U
-  current block.
+  layers > l_dense: block relevance + top-C and sparse attention over sinks U blocks U
+  current block (one fused launch per layer, or two calls).
 A block-entry step refreshes the block means of every sparse layer (and, for the
 comparison, runs the dense full refresh).
 
@@ -25,10 +25,14 @@ from .configs import FocusConfig
 
 class SparseStep:
     def __init__(self, cfg: FocusConfig, Q_full: torch.Tensor, K: List[torch.Tensor], V: List[torch.Tensor],
-                 device="cuda"):
-        """Q_full [n_layers, B, Hq, L, d]; K[l], V[l] [B, Hkv, L, d] (bf16, on `device`)."""
+                 device="cuda", fused: bool = True):
+        """Q_full [n_layers, B, Hq, L, d]; K[l], V[l] [B, Hkv, L, d] (bf16, on `device`).
+
+        fused: each sparse layer runs block relevance + top-C and the sparse attention as
+        one launch (focus_sparse_attention_fused), else as two calls."""
         c = cfg
         self.cfg = c
+        self.fused = fused
         self.dev = torch.device(device)
         self.Q_full, self.K, self.V = Q_full, K, V
         self.scale = 1.0 / math.sqrt(c.d)
@@ -121,8 +125,11 @@ class SparseStep:
         for l in range(min(c.l_dense + 1, c.n_layers)):
             timed("dense_attention" if l != c.l_dense else "dense_attention_colsum", self.dense_layer, l)
         for l in self.sparse_layers:
-            timed("block_select", self.block_select_layer, l)
-            timed("sparse_attention", self.sparse_attention_layer, l)
+            if self.fused:
+                timed("sparse_layer_fused", self.sparse_layer_fused, l)
+            else:
+                timed("block_select", self.block_select_layer, l)
+                timed("sparse_attention", self.sparse_attention_layer, l)
 
     # ------------------------------------------------------------------ graphs
     def capture(self):
