@@ -508,8 +508,11 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o, const floa
 // ------------------------------------------------------------------------- sink column sums
 // colsum[b, h, j] = sum over valid query rows r of the group of 2^(scale_log2 * q_r . k_j - lse2_r).
 // Swap-AB: S^T = K Q^T (M = 128 keys, N = padded group rows) so that each thread owns one
-// key and the sum over queries is thread-local.
-constexpr int kColStages = 3;
+// key and the sum over queries is thread-local. The S^T accumulator is double-buffered in
+// TMEM, so the MMA of tile i+1 overlaps the exp-sum of tile i. The K ring is as deep as
+// shared memory allows (6 stages for up to 64 group rows, else 3), because K is the only
+// stream and its bytes in flight bound the bandwidth.
+constexpr int kColMaxStages = 6;
 
 struct ColsumArgs {
   const __nv_bfloat16* Q;
@@ -524,29 +527,33 @@ struct ColsumArgs {
 };
 
 struct __align__(8) ColBook {
-  uint64_t full[kColStages];
-  uint64_t empty[kColStages];
-  uint64_t acc_full, acc_free, drain;
+  uint64_t full[kColMaxStages];
+  uint64_t empty[kColMaxStages];
+  uint64_t acc_full[2], acc_free[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   float lse2[256];
 };
 
-template <int D>
+template <int D, int STAGES>
 struct ColSmem {
+  static constexpr int kQRows = STAGES > 3 ? 64 : 256;     // group rows the Q area holds
   static constexpr uint32_t kTile = kBN * D * 2;
-  static constexpr uint32_t kQ = 0;                        // up to 256 rows
-  static constexpr uint32_t kK = kQ + 256 * D * 2;
-  static constexpr uint32_t kBook = kK + kColStages * kTile;
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kK = kQ + kQRows * D * 2;
+  static constexpr uint32_t kBook = kK + STAGES * kTile;
   static constexpr uint32_t kBytes = kBook + sizeof(ColBook) + 1024;
+  static_assert(STAGES <= kColMaxStages, "too many stages");
+  static_assert(kBytes <= 232448, "colsum kernel exceeds the 227 KB of shared memory per CTA");
 };
 
-template <int D>
+template <int D, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     colsum_kernel(const __grid_constant__ CUtensorMap tmK128, const ColsumArgs a) {
   griddep_wait();               // inputs may come from the previous kernel on the stream
   griddep_launch_dependents();
-  using SM = ColSmem<D>;
+  using SM = ColSmem<D, STAGES>;
+  constexpr int kColStages = STAGES;
   constexpr int CH = D / 8;
   constexpr int ATOMS = D / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -570,8 +577,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bk->full[s], 1);
       mbar_init(&bk->empty[s], 1);
     }
-    mbar_init(&bk->acc_full, 1);
-    mbar_init(&bk->acc_free, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bk->acc_full[i], 1);
+      mbar_init(&bk->acc_free[i], 4);
+    }
     mbar_init(&bk->drain, 1);
     bk->abort_flag = 0;
     fence_mbar_init();
@@ -632,17 +641,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_base = smem_u32(sQ);
       for (int it = 0; it < n_it; ++it) {
         const int s = it % kColStages;
+        const int ab = it & 1;
         if (!mbar_wait(&bk->full[s], (it / kColStages) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
-        if (it > 0 && !mbar_wait(&bk->acc_free, (it - 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
+        if (it >= 2 && !mbar_wait(&bk->acc_free[ab], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
+          break;
         tc_fence_after();
         const uint32_t k_base = smem_u32(sK + s * SM::kTile);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t da = sw128_desc(k_base + (ks >> 2) * (kBN * 128) + (ks & 3) * 32, 16, 1024);
           const uint64_t db = sw128_desc(q_base + (ks >> 2) * (n_pad * 128) + (ks & 3) * 32, 16, 1024);
-          mma_bf16(tmem, da, db, idesc, ks > 0 ? 1u : 0u);
+          mma_bf16(tmem + ab * n_pad, da, db, idesc, ks > 0 ? 1u : 0u);
         }
-        mma_commit(&bk->acc_full);
+        mma_commit(&bk->acc_full[ab]);
         mma_commit(&bk->empty[s]);
       }
       mma_commit(&bk->drain);
@@ -653,13 +664,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
     float* out = a.colsum + static_cast<size_t>(bh) * a.L;
     for (int it = 0; it < n_it; ++it) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&bk->acc_full, it & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE)))
+      const int ab = it & 1;
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&bk->acc_full[ab], (it >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE)))
         break;
       tc_fence_after();
       float sum = 0.f;
       for (int c0 = 0; c0 < n_pad; c0 += 32) {
         uint32_t rg[32];
-        tmem_ld32(tmem + lane_addr + c0, rg);
+        tmem_ld32(tmem + lane_addr + ab * n_pad + c0, rg);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -669,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bk->acc_free);
+      if (lane == 0) mbar_arrive(&bk->acc_free[ab]);
       const int key = (t_begin + it) * kBN + threadIdx.x;
       if (key < a.L) out[key] = sum;
     }
@@ -813,10 +826,10 @@ int launch_combine(const AttnArgs& a, cudaStream_t stream) {
   return FOCUS_OK;
 }
 
-template <int D>
+template <int D, int STAGES>
 int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const float* lse2, float* colsum,
                   int B, int Hq, int Hkv, int L, int qcap, float scale_log2, cudaStream_t stream) {
-  using SM = ColSmem<D>;
+  using SM = ColSmem<D, STAGES>;
   CUtensorMap mk;
   const int box_rows = box_rows_for(false, L, 0, 0);
   int st = make_kv_map(&mk, K, B * Hkv, L, D, box_rows);
@@ -834,7 +847,7 @@ int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat1
   c.qcap = qcap;
   c.g = Hq / Hkv;
   c.n_pad = ((c.g * qcap + 15) / 16) * 16;
-  c.tmem_cols = c.n_pad <= 32 ? 32 : c.n_pad <= 64 ? 64 : c.n_pad <= 128 ? 128 : 256;
+  c.tmem_cols = 2 * c.n_pad <= 32 ? 32 : 2 * c.n_pad <= 64 ? 64 : 2 * c.n_pad <= 128 ? 128 : 2 * c.n_pad <= 256 ? 256 : 512;
   c.scale_log2 = scale_log2;
   c.dev_err = device_error_word();
   const int total_tiles = (L + kBN - 1) / kBN;
@@ -844,7 +857,7 @@ int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat1
   chunks = std::min(chunks, total_tiles);
   c.tiles_per_cta = (total_tiles + chunks - 1) / chunks;
   chunks = (total_tiles + c.tiles_per_cta - 1) / c.tiles_per_cta;
-  auto kern = colsum_kernel<D>;
+  auto kern = colsum_kernel<D, STAGES>;
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SM::kBytes));
@@ -860,6 +873,16 @@ int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat1
   return FOCUS_OK;
 }
 
+// The deep ring needs the group rows to fit the 64-row Q area.
+template <int D>
+int run_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const float* lse2, float* colsum,
+               int B, int Hq, int Hkv, int L, int qcap, float scale_log2, cudaStream_t stream) {
+  const int n_pad = ((Hq / Hkv * qcap + 15) / 16) * 16;
+  if (n_pad <= ColSmem<D, 6>::kQRows)
+    return launch_colsum<D, 6>(Q, n_q, K, lse2, colsum, B, Hq, Hkv, L, qcap, scale_log2, stream);
+  return launch_colsum<D, 3>(Q, n_q, K, lse2, colsum, B, Hq, Hkv, L, qcap, scale_log2, stream);
+}
+
 template <int D, bool SPARSE>
 int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, cudaStream_t stream) {
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -869,7 +892,7 @@ int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, 
                               args.bs, args.P, args.g0, args.g1, SPARSE, args.B, args.Hq, args.Hkv, args.L, args.qcap,
                               args.scale_log2, stream);
     if (st == FOCUS_OK && colsum)
-      st = launch_colsum<D>(args.Q, args.n_q, args.K, lse, colsum, args.B, args.Hq, args.Hkv, args.L, args.qcap,
+      st = run_colsum<D>(args.Q, args.n_q, args.K, lse, colsum, args.B, args.Hq, args.Hkv, args.L, args.qcap,
                             args.scale_log2, stream);
     return st;
   }
@@ -900,7 +923,7 @@ int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, 
     if (st != FOCUS_OK) return st;
   }
   if (colsum) {
-    st = launch_colsum<D>(args.Q, args.n_q, args.K, args.lse_out, colsum, args.B, args.Hq, args.Hkv, args.L,
+    st = run_colsum<D>(args.Q, args.n_q, args.K, args.lse_out, colsum, args.B, args.Hq, args.Hkv, args.L,
                           args.qcap, args.scale_log2, stream);
   }
   return st;

@@ -79,6 +79,7 @@ struct __align__(8) DecBook {
   int blk[kDecMaxBlocks];
   int sinks[kDecMaxSinks];
   TopkShared tk;
+  uint64_t kb_bar;         // kbar rows staged by bulk copy (fused relevance prologue)
   uint32_t qvalid[2];      // bit q: query column q is a real query
   uint32_t tile_ctr;       // next dynamically claimed tile (CTA 0 of the cluster)
   int stage_tile[4];       // tile held by each ring stage, -1 = no more tiles
@@ -235,22 +236,35 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (!FUSED && cs > 1) cluster_arrive();
   if (FUSED) {
     // ---- block relevance R_b = qbar . kbar_b / sqrt(d) and top-C (method steps (4)) ----
-    // qbar over the active rows of this KV group; partial sums in the (still idle) K ring
+    // This CTA scores the contiguous kbar rows [j_begin, j_end). They are staged into the
+    // (still idle) V ring by bulk copies of up to kKbRound rows, the first issued before
+    // qbar is formed; qbar's partial sums use the (still idle) K ring.
+    constexpr int kKbRound = 128;
+    static_assert(kKbRound * D * 4 <= STAGES * SM::kTile, "kbar round exceeds the V ring");
     float* s_part = reinterpret_cast<float*>(sK);            // [3][D]
     float* s_qbar = s_part + 3 * D;                            // [D]
-    float* s_R = reinterpret_cast<float*>(sP);                 // [nb], every CTA holds all of R
+    float* s_kb = reinterpret_cast<float*>(sV);                // [kKbRound][D]
+    uint32_t* s_key = reinterpret_cast<uint32_t*>(sP);        // [nb] order keys of R, in every CTA
     const int rows = a.g * nq_b;
     const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
     const float* kb = a.kbar + static_cast<size_t>(bh) * a.nb * D;
     const int chunk = (a.nb + cs - 1) / cs;
-    const int j_begin = rank * chunk, j_end = min(a.nb, j_begin + chunk);
-    uint32_t* s_key = reinterpret_cast<uint32_t*>(s_R);
+    const int j_begin = min(a.nb, rank * chunk), j_end = min(a.nb, j_begin + chunk);
     const uint32_t sK0 = smem_u32(s_key);
+    auto issue_round = [&](int j0) {
+      const int nrow = min(kKbRound, j_end - j0);
+      mbar_arrive_expect_tx(&bk->kb_bar, static_cast<uint32_t>(nrow * D * 4));
+      bulk_load(smem_u32(s_kb), kb + static_cast<size_t>(j0) * D, static_cast<uint32_t>(nrow * D * 4), &bk->kb_bar);
+    };
+    if (threadIdx.x == 0) {
+      bk->abort_flag = 0;
+      mbar_init(&bk->kb_bar, 1);
+      fence_mbar_init();
+      if (j_begin < j_end) issue_round(j_begin);
+    }
     // qbar over the group's active rows: 3 row groups x 64 dim pairs, 8 rows in flight per
     // thread. Row slot r = (head r / qcap, position r % qcap); every slot is loaded and the
-    // positions >= nq_b are masked afterwards, so the loads do not wait for n_q. The first
-    // batch of Q rows is requested before this thread's first kbar row, so the
-    // latency-critical Q loads are not queued behind it.
+    // positions >= nq_b are masked afterwards, so the loads do not wait for n_q.
     const int t = threadIdx.x, dp = t % 64, rg = t / 64;
     const int nr = a.g * a.qcap;
     auto load8 = [&](int r0, __nv_bfloat162 (&v)[8]) {
@@ -274,16 +288,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (r - rh * a.qcap >= nq_b) v[u] = __floats2bfloat162_rn(0.f, 0.f);
       }
     };
-    __nv_bfloat162 qv8[8];
-    load8(rg, qv8);
-    int j = j_begin + threadIdx.x;
-    float4 kv[D / 4];
-    if (j < j_end) {
-      const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
-#pragma unroll
-      for (int c = 0; c < D / 4; ++c) kv[c] = __ldg(row + c);
-    }
     {
+      __nv_bfloat162 qv8[8];
+      load8(rg, qv8);
       float2 acc = make_float2(0.f, 0.f);
       for (int r0 = rg;;) {
         mask8(r0, qv8);
@@ -306,27 +313,36 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       s_qbar[threadIdx.x] = rows > 0 ? q / static_cast<float>(rows) : 0.f;
     }
     __syncthreads();
-    // R of this CTA's share of the blocks, one kbar row per thread; the order key of every
-    // score is broadcast to each CTA of the cluster
-    while (j < j_end) {
-      float p = 0.f;
+    // R of the staged rows: warp w scores groups of 32 rows, lane l holding dims
+    // 4l .. 4l+3 of every row of the group; a warp reduce-scatter leaves row g*32 + l's
+    // score in lane l. The order key of every score is broadcast to each CTA.
+    const float4 qv = reinterpret_cast<const float4*>(s_qbar)[lane];
+    for (int j0 = j_begin, round = 0; j0 < j_end; j0 += kKbRound, ++round) {
+      const int nrow = min(kKbRound, j_end - j0);
+      mbar_wait(&bk->kb_bar, round & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_PRODUCER);
+      for (int g0 = warp * 32; g0 < nrow; g0 += kDecThreads) {
+        float part[32];
 #pragma unroll
-      for (int c = 0; c < D / 4; ++c) {
-        const float4 qv = reinterpret_cast<const float4*>(s_qbar)[c];
-        p += qv.x * kv[c].x + qv.y * kv[c].y + qv.z * kv[c].z + qv.w * kv[c].w;
+        for (int r = 0; r < 32; ++r) {
+          const float4 kv = reinterpret_cast<const float4*>(s_kb + static_cast<size_t>(g0 + r) * D)[lane];
+          part[r] = (qv.x * kv.x + qv.y * kv.y) + (qv.z * kv.z + qv.w * kv.w);
+        }
+        warp_sum_scatter<32>(part);
+        if (g0 + lane < nrow) {
+          const int j = j0 + g0 + lane;
+          const uint32_t key = float_order_key(part[0] * inv_sqrt_d);
+          if (cs > 1) {
+            for (int r = 0; r < cs; ++r)
+              asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dsmem_addr(sK0 + 4u * j, r)), "r"(key)
+                           : "memory");
+          } else {
+            s_key[j] = key;
+          }
+        }
       }
-      const uint32_t key = float_order_key(p * inv_sqrt_d);
-      if (cs > 1) {
-        for (int r = 0; r < cs; ++r)
-          asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dsmem_addr(sK0 + 4u * j, r)), "r"(key) : "memory");
-      } else {
-        s_key[j] = key;
-      }
-      j += kDecThreads;
-      if (j < j_end) {
-        const float4* row = reinterpret_cast<const float4*>(kb + static_cast<size_t>(j) * D);
-#pragma unroll
-        for (int c = 0; c < D / 4; ++c) kv[c] = __ldg(row + c);
+      if (j0 + kKbRound < j_end) {
+        __syncthreads();               // every warp is done with this round's rows
+        if (threadIdx.x == 0) issue_round(j0 + kKbRound);
       }
     }
     if (cs > 1) cluster_sync();   // every CTA holds all nb keys
@@ -352,7 +368,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mbar_init(&bk->pv_done[i], 1);
       }
       mbar_init(&bk->drain, 1);
-      bk->abort_flag = 0;
+      if (!FUSED) bk->abort_flag = 0;   // the relevance prologue set it already
       fence_mbar_init();
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
