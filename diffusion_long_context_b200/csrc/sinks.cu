@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(kSinkThreads) sink_topk_regs_kernel(const floa
 // selection over the whole row. After a cluster barrier CTA 0 selects the top-S of the
 // cs * S candidates.
 template <int KPT>
-__global__ void __launch_bounds__(kSinkThreads) sink_topk_cluster_kernel(const float* __restrict__ colsum, int L,
+__global__ void __launch_bounds__(kSinkThreads, 2) sink_topk_cluster_kernel(const float* __restrict__ colsum, int L,
                                                                          int S, int chunk,
                                                                          int32_t* __restrict__ sinks, int vec) {
   griddep_wait();               // inputs may come from the previous kernel on the stream
@@ -148,10 +148,10 @@ extern "C" int focus_sink_identify(const float* colsum, int B, int Hkv, int L, i
   FOCUS_CHECK_ARG(B >= 0 && Hkv >= 1 && L >= 1 && S >= 1 && S <= 4096, "bad sizes (L=%d S=%d)", L, S);
   if (B == 0) return FOCUS_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // cluster form: cs CTAs per (b, h) while the grid fits the SMs and every share holds at
-  // least S columns and at most 16 per thread
+  // cluster form: cs CTAs per (b, h) while two CTAs per SM cover the grid and every share
+  // holds at least S columns and at most 16 per thread
   int cs = 1;
-  while (cs < 8 && B * Hkv * cs * 2 <= device_sm_count() && L >= cs * 2 * S && cs * 2 * S <= 4 * kSinkThreads)
+  while (cs < 8 && B * Hkv * cs * 2 <= 2 * device_sm_count() && L >= cs * 2 * S && cs * 2 * S <= 4 * kSinkThreads)
     cs *= 2;
   if (cs > 1 && (L + cs - 1) / cs <= 16 * kSinkThreads) {
     const int chunk = ((L + cs - 1) / cs + 3) & ~3;
