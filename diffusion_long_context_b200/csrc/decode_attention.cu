@@ -703,59 +703,75 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     tmem_dealloc(tmem, SM::kTmemCols);
   }
   const int qpc = (n_rows + cs - 1) / cs;
+  // lane: dims 4*lane .. 4*lane+3; warp: queries rank*qpc + warp + 4k, two per batch. A
+  // batch's partials are all requested before any is used; after its last batch a warp
+  // arrives on the cluster barrier (its reads are done) and waits on it only at the end.
+  const uint32_t po = smem_u32(part_o), pm = smem_u32(part_ml);
+  auto load_q = [&](int q, bool v, float4 (&ov)[8], float2 (&ml)[8]) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      ov[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      ml[r] = make_float2(-INFINITY, 0.f);
+      if (v && r < cs) {
+        ml[r] = dsmem_ld_v2(dsmem_addr(pm + static_cast<uint32_t>(q) * 8u, r));
+        ov[r] = dsmem_ld_v4(dsmem_addr(po + static_cast<uint32_t>(q * D + 4 * lane) * 4u, r));
+      }
+    }
+  };
+  auto finish_q = [&](int q, const float4 (&ov)[8], const float2 (&ml)[8]) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (ml[r].y > 0.f) M = fmaxf(M, ml[r].x);
+    float l = 0.f, w[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      w[r] = ml[r].y > 0.f ? exp2_approx(ml[r].x - M) : 0.f;
+      l += w[r] * ml[r].y;
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float wr = w[r] * inv;
+      o.x += wr * ov[r].x;
+      o.y += wr * ov[r].y;
+      o.z += wr * ov[r].z;
+      o.w += wr * ov[r].w;
+    }
+    const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
+    const int hq = kvh * a.g + qh, i = q - qh * a.qcap;
+    if (i >= nq_b) o = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint2 pk;
+    pk.x = pack_bf16x2(o.x, o.y);
+    pk.y = pack_bf16x2(o.z, o.w);
+    const size_t row = (static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i;
+    *reinterpret_cast<uint2*>(a.O + row * D + 4 * lane) = pk;
+    if (lane == 0 && a.lse_out && i < nq_b) a.lse_out[row] = M + __log2f(l);
+  };
+  bool arrived = false;
   if (warp < 4) {
-    // lane: dims 4*lane .. 4*lane+3; warp: queries rank*qpc + warp + 4k
-    const uint32_t po = smem_u32(part_o), pm = smem_u32(part_ml);
-    for (int qi = warp; qi < qpc; qi += 4) {
-      const int q = rank * qpc + qi;
-      if (q >= n_rows) break;
-      float4 ov[8];
-      float2 ml[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        ov[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-        ml[r] = make_float2(-INFINITY, 0.f);
-        if (r < cs) {
-          ml[r] = dsmem_ld_v2(dsmem_addr(pm + static_cast<uint32_t>(q) * 8u, r));
-          ov[r] = dsmem_ld_v4(dsmem_addr(po + static_cast<uint32_t>(q * D + 4 * lane) * 4u, r));
-        }
+    for (int qi0 = warp; qi0 < qpc; qi0 += 8) {
+      const int qa = rank * qpc + qi0, qb = qa + 4;
+      const bool va = qa < n_rows, vb = (qi0 + 4 < qpc) && qb < n_rows;
+      float4 ova[8], ovb[8];
+      float2 mla[8], mlb[8];
+      load_q(qa, va, ova, mla);
+      load_q(qb, vb, ovb, mlb);
+      if (cs > 1 && qi0 + 8 >= qpc) {
+        cluster_arrive();              // this warp's reads of the partials are done
+        arrived = true;
       }
-      float M = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (ml[r].y > 0.f) M = fmaxf(M, ml[r].x);
-      float l = 0.f, w[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        w[r] = ml[r].y > 0.f ? exp2_approx(ml[r].x - M) : 0.f;
-        l += w[r] * ml[r].y;
-      }
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const float wr = w[r] * inv;
-        o.x += wr * ov[r].x;
-        o.y += wr * ov[r].y;
-        o.z += wr * ov[r].z;
-        o.w += wr * ov[r].w;
-      }
-      const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
-      const int hq = kvh * a.g + qh, i = q - qh * a.qcap;
-      if (i >= nq_b) o = make_float4(0.f, 0.f, 0.f, 0.f);
-      uint2 pk;
-      pk.x = pack_bf16x2(o.x, o.y);
-      pk.y = pack_bf16x2(o.z, o.w);
-      const size_t row = (static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i;
-      *reinterpret_cast<uint2*>(a.O + row * D + 4 * lane) = pk;
-      if (lane == 0 && a.lse_out && i < nq_b) a.lse_out[row] = M + __log2f(l);
+      if (va) finish_q(qa, ova, mla);
+      if (vb) finish_q(qb, ovb, mlb);
     }
   }
   if (cs > 1) {
-    cluster_arrive();                // this CTA's reads of the partials are done
+    if (!arrived) cluster_arrive();
     cluster_wait();                  // no CTA leaves while its partials may still be read
   }
 }
+
 // ------------------------------------------------------------------------- host side
 namespace {
 

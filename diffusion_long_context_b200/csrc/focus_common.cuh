@@ -262,17 +262,18 @@ __device__ __forceinline__ uint32_t dsmem_atomic_add(uint32_t local_saddr, uint3
                : "memory");
   return old;
 }
+// Vector loads from a peer's shared memory. No memory clobber: several can be in flight;
+// they stay ordered with the (volatile) cluster barriers around them.
 __device__ __forceinline__ float4 dsmem_ld_v4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
+               : "r"(addr));
   return v;
 }
 __device__ __forceinline__ float2 dsmem_ld_v2(uint32_t addr) {
   float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
+  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
