@@ -261,18 +261,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kBM, D, false, true);
-      const uint32_t q_base = smem_u32(sQ), p_base = smem_u32(sP);
+      // Descriptors are formed once; a K step or a stage adds a constant to the 14-bit
+      // start-address field (address >> 4), which cannot carry: shared memory < 256 KB.
+      const uint64_t q_desc = sw128_desc(smem_u32(sQ), 16, 1024);
+      const uint64_t p_desc = sw128_desc(smem_u32(sP), 16, 1024);
+      const uint64_t k_desc0 = sw128_desc(smem_u32(sK), 16, 1024);
+      const uint64_t v_desc0 = sw128_desc(smem_u32(sV), kBN * 128, 1024);
+      constexpr uint32_t kTileDesc = SM::kTile >> 4;
       bool ok = true;
       auto issue_pv = [&](int j) -> bool {
         if (!mbar_wait(&bk->p_full, j & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t v_base = smem_u32(sV + (j % kStages) * SM::kTile);
+        const uint64_t vd = v_desc0 + static_cast<uint64_t>((j % kStages) * kTileDesc);
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks) {
-          const uint64_t da = sw128_desc(p_base + (ks >> 2) * (kBM * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t db = sw128_desc(v_base + ks * 2048, kBN * 128, 1024);
-          mma_bf16(tO, da, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kBN / 16; ++ks)
+          mma_bf16(tO, p_desc + (ks >> 2) * (kBM * 128 / 16) + (ks & 3) * 2, vd + ks * (2048 / 16), idesc_pv,
+                   (j > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bk->pv_done);
         mma_commit(&bk->empty[j % kStages]);
         return true;
@@ -282,13 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&bk->full[s], (it / kStages) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
         if (it > 0 && !mbar_wait(&bk->s_free, (it - 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + s * SM::kTile);
+        const uint64_t kd = k_desc0 + static_cast<uint64_t>(s * kTileDesc);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks >> 2) * (kBN * 128) + (ks & 3) * 32;
-          const uint64_t da = sw128_desc(q_base + koff, 16, 1024);
-          const uint64_t db = sw128_desc(k_base + koff, 16, 1024);
-          mma_bf16(tS, da, db, idesc_qk, ks > 0 ? 1u : 0u);
+          const uint32_t koff = (ks >> 2) * (kBN * 128 / 16) + (ks & 3) * 2;
+          mma_bf16(tS, q_desc + koff, kd + koff, idesc_qk, ks > 0 ? 1u : 0u);
         }
         mma_commit(&bk->s_full);
         if (it > 0) ok = issue_pv(it - 1);
@@ -638,7 +640,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(kBM, n_pad, false, false);
-      const uint32_t q_base = smem_u32(sQ);
+      // descriptors formed once; K steps and stages add constants to the start-address field
+      const uint64_t q_desc = sw128_desc(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc0 = sw128_desc(smem_u32(sK), 16, 1024);
       for (int it = 0; it < n_it; ++it) {
         const int s = it % kColStages;
         const int ab = it & 1;
@@ -646,13 +650,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it >= 2 && !mbar_wait(&bk->acc_free[ab], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
           break;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + s * SM::kTile);
+        const uint64_t kd = k_desc0 + static_cast<uint64_t>(s * (SM::kTile >> 4));
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t da = sw128_desc(k_base + (ks >> 2) * (kBN * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t db = sw128_desc(q_base + (ks >> 2) * (n_pad * 128) + (ks & 3) * 32, 16, 1024);
-          mma_bf16(tmem + ab * n_pad, da, db, idesc, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_bf16(tmem + ab * n_pad, kd + (ks >> 2) * (kBN * 128 / 16) + (ks & 3) * 2,
+                   q_desc + (ks >> 2) * (n_pad * 128 / 16) + (ks & 3) * 2, idesc, ks > 0 ? 1u : 0u);
         mma_commit(&bk->acc_full[ab]);
         mma_commit(&bk->empty[s]);
       }

@@ -481,21 +481,25 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_bf16_f32(128, NQ, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(128, NQ, true, false);
-      const uint32_t q_base = smem_u32(sQ);
       const uint32_t tO = tmem + 2 * NQ;
+      // Descriptors are formed once; a K step or a stage adds a constant to the 14-bit
+      // start-address field (address >> 4), which cannot carry: shared memory < 256 KB.
+      const uint64_t q_desc = sw128_desc(smem_u32(sQ), 16, 1024);
+      const uint64_t k_desc0 = sw128_desc(smem_u32(sK), 16, 1024);
+      const uint64_t v_desc0 = sw128_desc(smem_u32(sV), 128 * 128, 1024);
+      const uint64_t p_desc0 = sw128_desc(smem_u32(sP), 16, 1024);
+      constexpr uint32_t kTileDesc = SM::kTile >> 4;
       bool ok = true;
       auto issue_pv = [&](int j) -> bool {
         const int pb = j & 1;
         if (!mbar_wait(&bk->p_full[pb], (j >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) return false;
         tc_fence_after();
-        const uint32_t v_base = smem_u32(sV + (j % STAGES) * SM::kTile);
-        const uint32_t p_base = smem_u32(sP + pb * (NQ * 256));
+        const uint64_t vd = v_desc0 + static_cast<uint64_t>((j % STAGES) * kTileDesc);
+        const uint64_t pd = p_desc0 + static_cast<uint64_t>(pb * (NQ * 256 / 16));
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t da = sw128_desc(v_base + ks * 2048, 128 * 128, 1024);
-          const uint64_t db = sw128_desc(p_base + (ks >> 2) * (NQ * 128) + (ks & 3) * 32, 16, 1024);
-          mma_bf16(tO, da, db, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16(tO, vd + ks * (2048 / 16), pd + (ks >> 2) * (NQ * 128 / 16) + (ks & 3) * 2, idesc_pv,
+                   (j > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&bk->pv_done[pb]);
         mma_commit(&bk->empty[j % STAGES]);
         return true;
@@ -514,13 +518,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         if (it >= 2 && !mbar_wait(&bk->s_free[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
           break;
         tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + s * SM::kTile);
+        const uint64_t kd = k_desc0 + static_cast<uint64_t>(s * kTileDesc);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t da = sw128_desc(k_base + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
-          const uint64_t db = sw128_desc(q_base + (ks >> 2) * (NQ * 128) + (ks & 3) * 32, 16, 1024);
-          mma_bf16(tmem + sb * NQ, da, db, idesc_qk, ks > 0 ? 1u : 0u);
-        }
+        for (int ks = 0; ks < D / 16; ++ks)
+          mma_bf16(tmem + sb * NQ, kd + (ks >> 2) * (128 * 128 / 16) + (ks & 3) * 2,
+                   q_desc + (ks >> 2) * (NQ * 128 / 16) + (ks & 3) * 2, idesc_qk, ks > 0 ? 1u : 0u);
         mma_commit(&bk->s_full[sb]);
         if (it > 0) ok = issue_pv(it - 1);
       }
