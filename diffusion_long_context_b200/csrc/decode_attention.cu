@@ -504,19 +504,28 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mma_commit(&bk->empty[j % STAGES]);
         return true;
       };
-      for (int it = 0; ok; ++it) {
+      // QK runs one tile ahead of PV: QK(j + 1) only needs the S buffer that softmax(j - 1)
+      // has already read, so it is issued before PV(j), which waits for softmax(j)'s P.
+      // (Two tiles ahead would hold PV(j) behind the load of tile j + 2, whose ring stage
+      // is only freed by PV(j - 1): the loads in flight would shrink to one tile.)
+      constexpr int LA = 1;
+      int q_next = 0, n_end = -1;          // next QK tile; tile index of the end marker
+      // QK of tile it; at the end marker, releases the softmax warps and returns false
+      auto issue_qk = [&](int it) -> bool {
         const int s = it % STAGES, sb = it & 1;
-        if (!mbar_wait(&bk->full[s], (it / STAGES) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
-        if (bk->stage_tile[s] < 0) {
-          // end marker: release the softmax warps (they wait for the last PV's completion
-          // on pv_done), then finish the last tile
-          n_it = it;
-          mbar_arrive(&bk->s_full[sb]);
-          if (it > 0) ok = issue_pv(it - 1);
-          break;
+        if (!mbar_wait(&bk->full[s], (it / STAGES) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) {
+          ok = false;
+          return false;
         }
-        if (it >= 2 && !mbar_wait(&bk->s_free[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
-          break;
+        if (bk->stage_tile[s] < 0) {
+          n_end = it;
+          mbar_arrive(&bk->s_full[sb]);
+          return false;
+        }
+        if (it >= 2 && !mbar_wait(&bk->s_free[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) {
+          ok = false;
+          return false;
+        }
         tc_fence_after();
         const uint64_t kd = k_desc0 + static_cast<uint64_t>(s * kTileDesc);
 #pragma unroll
@@ -524,8 +533,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           mma_bf16(tmem + sb * NQ, kd + (ks >> 2) * (128 * 128 / 16) + (ks & 3) * 2,
                    q_desc + (ks >> 2) * (NQ * 128 / 16) + (ks & 3) * 2, idesc_qk, ks > 0 ? 1u : 0u);
         mma_commit(&bk->s_full[sb]);
-        if (it > 0) ok = issue_pv(it - 1);
+        return true;
+      };
+      while (q_next < LA && n_end < 0 && ok && issue_qk(q_next)) ++q_next;
+      for (int j = 0; ok; ++j) {
+        if (n_end >= 0 && j >= n_end) break;
+        if (n_end < 0 && issue_qk(q_next)) ++q_next;
+        if (!ok) break;
+        ok = issue_pv(j);
       }
+      n_it = max(n_end, 0);
       mma_commit(&bk->drain);
       dec_wait_drain(&bk->drain, 0);
     }
