@@ -21,8 +21,9 @@
 // contiguous share of the key tiles, and the partial results (m, l, O) are merged through
 // distributed shared memory -- no workspace and no second launch.
 //
-// Warps: 0-3 softmax / epilogue, 4 producer (TMA for key runs, cp.async for sink rows),
-// 5 tcgen05.mma issuer and TMEM owner. K/V tiles flow through a STAGES-deep ring.
+// Warps: 0-7 softmax / epilogue (two per TMEM lane quadrant, each taking half of the
+// query columns), 8 producer (TMA for key runs, cp.async for sink rows), 9 tcgen05.mma
+// issuer and TMEM owner. K/V tiles flow through a STAGES-deep ring.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -37,12 +38,14 @@
 
 namespace focus {
 
-constexpr int kDecThreads = 192;
+constexpr int kDecSoftmaxWarps = 8;   // two per TMEM lane quadrant, each half of the queries
+constexpr int kDecSoftmaxThreads = kDecSoftmaxWarps * 32;
+constexpr int kDecThreads = kDecSoftmaxThreads + 64;
 constexpr int kDecD = 128;
 constexpr int kDecMaxBlocks = 512;
 constexpr int kDecMaxSinks = 512;
-constexpr int kDecProducerWarp = 4;
-constexpr int kDecMmaWarp = 5;
+constexpr int kDecProducerWarp = kDecSoftmaxWarps;
+constexpr int kDecMmaWarp = kDecSoftmaxWarps + 1;
 
 struct DecArgs {
   const __nv_bfloat16* Q;      // [B, Hq, qcap, D]
@@ -241,8 +244,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // qbar is formed; qbar's partial sums use the (still idle) K ring.
     constexpr int kKbRound = 128;
     static_assert(kKbRound * D * 4 <= STAGES * SM::kTile, "kbar round exceeds the V ring");
-    float* s_part = reinterpret_cast<float*>(sK);            // [3][D]
-    float* s_qbar = s_part + 3 * D;                            // [D]
+    constexpr int RG = kDecThreads / 64;                       // qbar row groups
+    float* s_part = reinterpret_cast<float*>(sK);            // [RG][D]
+    float* s_qbar = s_part + RG * D;                           // [D]
     float* s_kb = reinterpret_cast<float*>(sV);                // [kKbRound][D]
     uint32_t* s_key = reinterpret_cast<uint32_t*>(sP);        // [nb] order keys of R, in every CTA
     const int rows = a.g * nq_b;
@@ -262,7 +266,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       fence_mbar_init();
       if (j_begin < j_end) issue_round(j_begin);
     }
-    // qbar over the group's active rows: 3 row groups x 64 dim pairs, 8 rows in flight per
+    // qbar over the group's active rows: RG row groups x 64 dim pairs, 8 rows in flight per
     // thread. Row slot r = (head r / qcap, position r % qcap); every slot is loaded and the
     // positions >= nq_b are masked afterwards, so the loads do not wait for n_q.
     const int t = threadIdx.x, dp = t % 64, rg = t / 64;
@@ -270,7 +274,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     auto load8 = [&](int r0, __nv_bfloat162 (&v)[8]) {
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int r = r0 + 3 * u;
+        const int r = r0 + RG * u;
         v[u] = __floats2bfloat162_rn(0.f, 0.f);
         if (r < nr) {
           const int rh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
@@ -283,7 +287,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     auto mask8 = [&](int r0, __nv_bfloat162 (&v)[8]) {
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int r = r0 + 3 * u;
+        const int r = r0 + RG * u;
         const int rh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
         if (r - rh * a.qcap >= nq_b) v[u] = __floats2bfloat162_rn(0.f, 0.f);
       }
@@ -300,7 +304,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           acc.x += f.x;
           acc.y += f.y;
         }
-        r0 += 3 * 8;
+        r0 += RG * 8;
         if (r0 >= nr) break;
         load8(r0, qv8);
       }
@@ -309,7 +313,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     __syncthreads();
     if (threadIdx.x < D) {
-      const float q = (s_part[threadIdx.x] + s_part[D + threadIdx.x]) + s_part[2 * D + threadIdx.x];
+      float q = 0.f;
+#pragma unroll
+      for (int g = 0; g < RG; ++g) q += s_part[g * D + threadIdx.x];
       s_qbar[threadIdx.x] = rows > 0 ? q / static_cast<float>(rows) : 0.f;
     }
     __syncthreads();
@@ -363,8 +369,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
       for (int i = 0; i < 2; ++i) {
         mbar_init(&bk->s_full[i], 1);
-        mbar_init(&bk->s_free[i], 4);
-        mbar_init(&bk->p_full[i], 4);
+        mbar_init(&bk->s_free[i], kDecSoftmaxWarps);
+        mbar_init(&bk->p_full[i], kDecSoftmaxWarps);
         mbar_init(&bk->pv_done[i], 1);
       }
       mbar_init(&bk->drain, 1);
@@ -406,7 +412,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (warp != kDecProducerWarp) {
     // Q rows (query q <-> head kvh*g + q/qcap, position q%qcap) as a K-major SW128 B
     // operand; rows are loaded before the valid count is known and masked afterwards
-    const int qt = warp < kDecProducerWarp ? threadIdx.x : threadIdx.x - 32;   // 0..159 without the producer
+    const int qt = warp < kDecProducerWarp ? threadIdx.x : threadIdx.x - 32;   // dense index without the producer
     for (int idx = qt; idx < NQ * CH; idx += kDecThreads - 32) {
       const int q = idx / CH, c = idx % CH;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -440,9 +446,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const uint32_t tmem = bk->tmem_base;
   const SlotLayout sl = bk->sl;
   int n_it = 0;                                  // tiles this CTA processed (set by each role)
-  float lsum[NQ];
+  constexpr int QH = NQ / 2;                     // query columns per softmax thread
+  float lsum[QH];
 #pragma unroll
-  for (int q = 0; q < NQ; ++q) lsum[q] = 0.f;
+  for (int q = 0; q < QH; ++q) lsum[q] = 0.f;
 
   if (warp == kDecProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -548,14 +555,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warps 0..3
-    const int t = threadIdx.x;                         // key of the tile == TMEM lane == dim of O^T
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    // ------------------------------------------------------------ softmax warps 0..7
+    // Warp w reads TMEM lane quadrant w % 4 (keys 32*(w%4) .. +31 of the tile, or dims of
+    // O^T) and query half w / 4 (columns q0 .. q0 + QH - 1).
+    const int t = threadIdx.x & 127;                   // key of the tile == TMEM lane == dim of O^T
+    const int qd = warp & 3;
+    const int q0 = (warp >> 2) * QH;
+    const uint32_t lane_addr = static_cast<uint32_t>(qd * 32) << 16;
     const uint32_t tO = tmem + 2 * NQ;
-    const uint64_t qvalid = bk->qvalid[0] | (static_cast<uint64_t>(bk->qvalid[1]) << 32);
-    // The loop ends, in all four warps at once, at the end marker or when a wait ran out.
+    const uint64_t qvalid =
+        (bk->qvalid[0] | (static_cast<uint64_t>(bk->qvalid[1]) << 32)) >> q0;   // bit q: column q0 + q is real
+    // The loop ends, in all eight warps at once, at the end marker or when a wait ran out.
     // A warp whose wait ran out inside an iteration finishes it without waits or
-    // tensor-memory access, so that all four warps take the same named-barrier steps.
+    // tensor-memory access, so that all eight warps take the same named-barrier steps.
     bool ok = true;
     int it = 0;
     for (;; ++it) {
@@ -570,20 +582,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                                DEV_ERR_TIMEOUT_SOFTMAX));
         if (ok) tile = bk->stage_tile[it % STAGES];
       }
-      if (bar_red_or(1, 128, tile < 0 || *abort_flag != 0)) break;
-      float sv[NQ];
+      if (bar_red_or(1, kDecSoftmaxThreads, tile < 0 || *abort_flag != 0)) break;
+      float sv[QH];
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) sv[q] = 0.f;
+      for (int q = 0; q < QH; ++q) sv[q] = 0.f;
       if (ok) {
         tc_fence_after();
+        uint32_t rg[QH];
+        tmem_ld_cols<QH>(tmem + lane_addr + sb * NQ + q0, rg);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < NQ / 32; ++c) {
-          uint32_t rg[32];
-          tmem_ld32(tmem + lane_addr + sb * NQ + c * 32, rg);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) sv[c * 32 + j] = __uint_as_float(rg[j]);
-        }
+        for (int q = 0; q < QH; ++q) sv[q] = __uint_as_float(rg[q]);
       }
       tc_fence_before();
       __syncwarp();
@@ -591,63 +600,62 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const bool kv = ok && slot_valid<SPARSE>(sl, a.L, a.bs, G, tile * 128 + t);
       bool over = false;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
+      for (int q = 0; q < QH; ++q) {
         sv[q] = (kv && ((qvalid >> q) & 1ull)) ? sv[q] * a.scale_log2 : -INFINITY;
-        over |= sv[q] > bk->mref[q] + 8.f;
+        over |= sv[q] > bk->mref[q0 + q] + 8.f;
       }
-      if (bar_red_or(1, 128, over)) {
+      if (bar_red_or(1, kDecSoftmaxThreads, over)) {
         // exact per-query maximum of this tile, then move the references up
         // (one redux per query on the order-preserving integer image of the score)
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
+        for (int q = 0; q < QH; ++q) {
           const uint32_t m = __reduce_max_sync(0xffffffffu, float_order_key(sv[q]));
-          if (lane == 0) bk->red[warp][q] = __uint_as_float(m);
+          if (lane == 0) bk->red[qd][q0 + q] = __uint_as_float(m);
         }
-        named_bar_sync(1, 128);
-        if (t < NQ) {
-          const uint32_t k01 = max(__float_as_uint(bk->red[0][t]), __float_as_uint(bk->red[1][t]));
-          const uint32_t k23 = max(__float_as_uint(bk->red[2][t]), __float_as_uint(bk->red[3][t]));
+        named_bar_sync(1, kDecSoftmaxThreads);
+        if (threadIdx.x < NQ) {
+          const int tq = threadIdx.x;
+          const uint32_t k01 = max(__float_as_uint(bk->red[0][tq]), __float_as_uint(bk->red[1][tq]));
+          const uint32_t k23 = max(__float_as_uint(bk->red[2][tq]), __float_as_uint(bk->red[3][tq]));
           const float mt = order_key_to_float(max(k01, k23));
-          const float mo = bk->mref[t];
+          const float mo = bk->mref[tq];
           const float mn = fmaxf(mo, mt);
           if (mn > mo + 8.f || (mo == -INFINITY && mn > -INFINITY)) {
-            bk->alpha[t] = (mo == -INFINITY) ? 0.f : exp2_approx(mo - mn);
-            bk->mref[t] = mn;
+            bk->alpha[tq] = (mo == -INFINITY) ? 0.f : exp2_approx(mo - mn);
+            bk->mref[tq] = mn;
           } else {
-            bk->alpha[t] = 1.f;
+            bk->alpha[tq] = 1.f;
           }
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(1, kDecSoftmaxThreads);
         bool any_scale = false;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const float al = bk->alpha[q];
+        for (int q = 0; q < QH; ++q) {
+          const float al = bk->alpha[q0 + q];
           lsum[q] *= al;
           any_scale |= al != 1.f;
         }
+        any_scale = __any_sync(0xffffffffu, any_scale);
         if (it > 0 && any_scale && ok) {
           // O^T must hold PV of the previous tile before it is rescaled
           ok = __all_sync(0xffffffffu, mbar_wait(&bk->pv_done[(it - 1) & 1], ((it - 1) >> 1) & 1, abort_flag,
                                                  a.dev_err, DEV_ERR_TIMEOUT_SOFTMAX));
           if (ok) {
             tc_fence_after();
+            uint32_t rg[QH];
+            tmem_ld_cols<QH>(tO + lane_addr + q0, rg);
+            tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < NQ / 32; ++c) {
-              uint32_t rg[32];
-              tmem_ld32(tO + lane_addr + c * 32, rg);
-              tmem_ld_wait();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) rg[j] = __float_as_uint(__uint_as_float(rg[j]) * bk->alpha[c * 32 + j]);
-              tmem_st32(tO + lane_addr + c * 32, rg);
-            }
+            for (int q = 0; q < QH; ++q) rg[q] = __float_as_uint(__uint_as_float(rg[q]) * bk->alpha[q0 + q]);
+            tmem_st_cols<QH>(tO + lane_addr + q0, rg);
             tmem_st_wait();
           }
         }
       }
       // P^T of this key: p = 2^(s - m_q)
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const float m = bk->mref[q];
+      for (int q = 0; q < QH; ++q) {
+        const float m = bk->mref[q0 + q];
         sv[q] = exp2_approx(sv[q] - (m == -INFINITY ? 0.f : m));
         lsum[q] += sv[q];
       }
@@ -658,9 +666,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         uint8_t* pbuf = sP + sb * (NQ * 256);
         const uint32_t col = static_cast<uint32_t>((t & 7) * 2);
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const __nv_bfloat16 h = __float2bfloat16_rn(sv[q]);
-          *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128_offset(q, t >> 3, NQ) + col) = h;
+        for (int q = 0; q < QH; ++q) {
+          const __nv_bfloat16 hv = __float2bfloat16_rn(sv[q]);
+          *reinterpret_cast<__nv_bfloat16*>(pbuf + sw128_offset(q0 + q, t >> 3, NQ) + col) = hv;
         }
         fence_proxy_async_smem();
       }
@@ -674,13 +682,21 @@ __global__ void __launch_bounds__(kDecThreads, 1)
                                              a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE));
       tc_fence_after();
     }
-    // row sums: reduce the per-key partials over the 128 threads (reduce-scatter per warp,
-    // then the four warps' sums; the epilogue's CTA barrier orders lfin)
-    warp_sum_scatter<NQ>(lsum);
+    // row sums: reduce the per-key partials over the 32 lanes of each warp (reduce-scatter),
+    // then over the four lane quadrants; the epilogue's CTA barrier orders lfin
+    if constexpr (QH % 32 == 0) {
+      warp_sum_scatter<QH>(lsum);
 #pragma unroll
-    for (int j = 0; j < NQ / 32; ++j) bk->red[warp][lane * (NQ / 32) + j] = lsum[j];
-    named_bar_sync(1, 128);
-    if (t < NQ) bk->lfin[t] = (bk->red[0][t] + bk->red[1][t]) + (bk->red[2][t] + bk->red[3][t]);
+      for (int j = 0; j < QH / 32; ++j) bk->red[qd][q0 + lane * (QH / 32) + j] = lsum[j];
+    } else {
+      warp_sum_scatter16(lsum);
+      if ((lane & 1) == 0) bk->red[qd][q0 + (lane >> 1)] = lsum[0];
+    }
+    named_bar_sync(1, kDecSoftmaxThreads);
+    if (threadIdx.x < NQ) {
+      const int tq = threadIdx.x;
+      bk->lfin[tq] = (bk->red[0][tq] + bk->red[1][tq]) + (bk->red[2][tq] + bk->red[3][tq]);
+    }
     if (!ok) bk->abort_flag = 1;
   }
 
@@ -697,20 +713,19 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   static_assert(NQ * D * 4 + NQ * 8 <= STAGES * SM::kTile, "partials exceed the V ring");
   float* part_o = reinterpret_cast<float*>(sV);                      // [NQ][D]
   float2* part_ml = reinterpret_cast<float2*>(part_o + NQ * D);      // [NQ] (m, l)
-  if (warp < 4) {
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+  if (warp < kDecSoftmaxWarps) {
+    // warp w: dims of lane quadrant w % 4, query half w / 4
+    const int t = threadIdx.x & 127, q0 = (warp >> 2) * QH;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t rg[QH];
 #pragma unroll
-    for (int c = 0; c < NQ / 32; ++c) {
-      uint32_t rg[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) rg[j] = 0u;
-      if (have_o) {
-        tmem_ld32(tmem + 2 * NQ + lane_addr + c * 32, rg);
-        tmem_ld_wait();
-      }
-#pragma unroll
-      for (int j = 0; j < 32; ++j) part_o[(c * 32 + j) * D + threadIdx.x] = __uint_as_float(rg[j]);
+    for (int j = 0; j < QH; ++j) rg[j] = 0u;
+    if (have_o) {
+      tmem_ld_cols<QH>(tmem + 2 * NQ + lane_addr + q0, rg);
+      tmem_ld_wait();
     }
+#pragma unroll
+    for (int j = 0; j < QH; ++j) part_o[(q0 + j) * D + t] = __uint_as_float(rg[j]);
     if (threadIdx.x < NQ)
       part_ml[threadIdx.x] = make_float2(bk->mref[threadIdx.x], have_o ? bk->lfin[threadIdx.x] : 0.f);
   }
@@ -722,7 +737,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     tmem_dealloc(tmem, SM::kTmemCols);
   }
   const int qpc = (n_rows + cs - 1) / cs;
-  // lane: dims 4*lane .. 4*lane+3; warp: queries rank*qpc + warp + 4k, two per batch. A
+  // lane: dims 4*lane .. 4*lane+3; warp: queries rank*qpc + warp + 8k, two per batch. A
   // batch's partials are all requested before any is used; after its last batch a warp
   // arrives on the cluster barrier (its reads are done) and waits on it only at the end.
   const uint32_t po = smem_u32(part_o), pm = smem_u32(part_ml);
@@ -769,15 +784,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (lane == 0 && a.lse_out && i < nq_b) a.lse_out[row] = M + __log2f(l);
   };
   bool arrived = false;
-  if (warp < 4) {
-    for (int qi0 = warp; qi0 < qpc; qi0 += 8) {
-      const int qa = rank * qpc + qi0, qb = qa + 4;
-      const bool va = qa < n_rows, vb = (qi0 + 4 < qpc) && qb < n_rows;
+  if (warp < kDecSoftmaxWarps) {
+    constexpr int W = kDecSoftmaxWarps;
+    for (int qi0 = warp; qi0 < qpc; qi0 += 2 * W) {
+      const int qa = rank * qpc + qi0, qb = qa + W;
+      const bool va = qa < n_rows, vb = (qi0 + W < qpc) && qb < n_rows;
       float4 ova[8], ovb[8];
       float2 mla[8], mlb[8];
       load_q(qa, va, ova, mla);
       load_q(qb, vb, ovb, mlb);
-      if (cs > 1 && qi0 + 8 >= qpc) {
+      if (cs > 1 && qi0 + 2 * W >= qpc) {
         cluster_arrive();              // this warp's reads of the partials are done
         arrived = true;
       }

@@ -356,6 +356,38 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+// N consecutive columns (N a multiple of 16) of this warp's 32 lanes into r (no wait).
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  static_assert(N % 16 == 0, "columns come in 16s");
+#pragma unroll
+  for (int c = 0; c < N / 32; ++c) tmem_ld32(taddr + c * 32, *reinterpret_cast<uint32_t(*)[32]>(r + c * 32));
+  if (N % 32) tmem_ld16(taddr + (N / 32) * 32, *reinterpret_cast<uint32_t(*)[16]>(r + (N / 32) * 32));
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  static_assert(N % 16 == 0, "columns come in 16s");
+#pragma unroll
+  for (int c = 0; c < N / 32; ++c)
+    tmem_st32(taddr + c * 32, *reinterpret_cast<const uint32_t(*)[32]>(r + c * 32));
+  if (N % 32) tmem_st16(taddr + (N / 32) * 32, *reinterpret_cast<const uint32_t(*)[16]>(r + (N / 32) * 32));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -418,7 +450,9 @@ __device__ __forceinline__ float order_key_to_float(uint32_t k) {
 
 // Warp reduce-scatter of N per-lane values (N a multiple of 32): afterwards v[j] of lane
 // l, j < N / 32, holds the sum over the 32 lanes of value index l * (N / 32) + j.
-// 31 * N / 32 shuffles instead of 5 * N for N separate butterfly sums.
+// 31 * N / 32 shuffles instead of 5 * N for N separate butterfly sums. For N = 16 the
+// halvings stop at one value per lane: lanes l and l ^ 1 then hold the two halves of
+// value index l >> 1 (warp_sum_scatter16 adds them).
 template <int N>
 __device__ __forceinline__ void warp_sum_scatter(float (&v)[N]) {
   const int lane = threadIdx.x & 31;
@@ -432,6 +466,12 @@ __device__ __forceinline__ void warp_sum_scatter(float (&v)[N]) {
       v[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
     }
   }
+}
+
+// v[0] of lane l = sum over the 32 lanes of value index l >> 1 (N = 16 values per lane).
+__device__ __forceinline__ void warp_sum_scatter16(float (&v)[16]) {
+  warp_sum_scatter<16>(v);
+  v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
 }
 
 #endif  // __CUDACC__
