@@ -151,9 +151,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
       const int32_t* blk_g = a.blocks + static_cast<size_t>(bh) * a.C;
       const int32_t* snk_g = a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr;
-      build_sparse_layout(layout_prefetch(blk_g, a.C, snk_g, a.S), blk_g, a.C, snk_g, a.S, a.L, a.P, a.bs, a.g0, a.g1,
-                          a.gen_pad, a.box_rows, a.pad_div, a.bs_div, bk->blk, kMaxBlocks, bk->fsinks, kMaxSinks,
-                          &bk->sl);
+      const LayoutPrefetch pf = layout_prefetch(blk_g, a.C, snk_g, a.S);
+      const SlotLayout sl0 = build_block_layout(pf, blk_g, a.C, a.S, a.P, a.bs, a.gen_pad, a.box_rows, a.pad_div,
+                                                bk->blk, kMaxBlocks, kMaxSinks, &bk->sl);
+      dedupe_sinks(pf, snk_g, sl0, a.L, a.P, a.g0, a.g1, a.bs_div, bk->blk, bk->fsinks);
     }
   } else if (threadIdx.x == 0) {
     bk->sl.n_slots = a.L;
@@ -326,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot0 = (t_begin + it) * kBN;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-          vm[q] = __ballot_sync(0xffffffffu, slot_valid<SPARSE>(sl, a.L, a.bs, a.g1 - a.g0, slot0 + q * 32 + lane));
+          vm[q] = __ballot_sync(0xffffffffu,
+                                slot_valid<SPARSE>(sl, bk->fsinks, a.L, a.bs, a.g1 - a.g0, slot0 + q * 32 + lane));
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t rg[32];

@@ -381,8 +381,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     if (SPARSE) {
       if (FUSED) pf = layout_prefetch(blk_g, a.C, snk_g, a.S);
-      sl_p = build_sparse_layout(pf, blk_g, a.C, snk_g, a.S, a.L, a.P, a.bs, a.g0, a.g1, a.gen_pad, a.box_rows,
-                                 a.pad_div, a.bs_div, bk->blk, kDecMaxBlocks, bk->sinks, kDecMaxSinks, &bk->sl);
+      sl_p = build_block_layout(pf, blk_g, a.C, a.S, a.P, a.bs, a.gen_pad, a.box_rows, a.pad_div, bk->blk,
+                                kDecMaxBlocks, kDecMaxSinks, &bk->sl);
     } else {
       sl_p.n_slots = a.L;
       if (lane == 0) bk->sl = sl_p;
@@ -392,6 +392,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // the layout and the barriers are ready: release the other warps, then fill the ring
     // (a tile gathered row by row completes after the TMA tiles behind it are issued)
     named_bar_arrive(2, kDecThreads);
+    // Tiles of kept blocks and of the current block do not need the sinks: they are issued
+    // first, and the sinks are de-duplicated just before the first tile that holds sink
+    // slots, at the latest before any tile beyond this first round.
+    bool sinks_ready = !SPARSE;
+    auto ensure_sinks = [&]() {
+      if (SPARSE && !sinks_ready) {
+        dedupe_sinks(pf, snk_g, sl_p, a.L, a.P, a.g0, a.g1, a.bs_div, bk->blk, bk->sinks);
+        sinks_ready = true;
+      }
+    };
     unsigned deferred = 0;
     for (int it = 0; it < STAGES; ++it) {
       const int tile = rank + it * cs;
@@ -400,8 +410,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         p_more = false;
         break;
       }
+      if (tile * 128 < sl_p.gen_start) ensure_sinks();
       if (produce(it, tile, true)) deferred |= 1u << it;
     }
+    ensure_sinks();
     if (deferred) finish_deferred(deferred);
     if (!FUSED && cs > 1) cluster_wait();   // the claim counter is initialised
   }
@@ -597,7 +609,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bk->s_free[sb]);
-      const bool kv = ok && slot_valid<SPARSE>(sl, a.L, a.bs, G, tile * 128 + t);
+      const bool kv = ok && slot_valid<SPARSE>(sl, bk->sinks, a.L, a.bs, G, tile * 128 + t);
       bool over = false;
 #pragma unroll
       for (int q = 0; q < QH; ++q) {

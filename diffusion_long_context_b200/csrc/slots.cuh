@@ -3,9 +3,10 @@
 // Dense: slot s is key s, s < L.
 // Sparse (Focus-dLLM method steps (5): I_p = sinks U kept prompt blocks U current
 // block, each key once): slots are laid out as
-//   [ de-duplicated sinks ]                sinks inside a kept block or the current
-//                                          block, out-of-range and repeated entries
-//                                          dropped; padded to a multiple of box_rows
+//   [ sinks ]                              one slot per listed sink; sinks inside a kept
+//                                          block or the current block, out-of-range and
+//                                          repeated entries are dropped (invalid slots);
+//                                          padded to a multiple of box_rows
 //   [ current block [g0, g1) ]             padded to gen_pad slots (a multiple of box_rows >= G)
 //   [ kept block 0 | kept block 1 | ... ]  each padded to pad_bs = round_up(bs, 8)
 // Padding slots are invalid (masked out of the softmax). Every box_rows-aligned group of
@@ -20,7 +21,7 @@ namespace focus {
 
 struct SlotLayout {
   int n_slots;      // total slots (keys + padding)
-  int n_fsinks;     // sinks that remain after de-duplication (slots [0, n_fsinks))
+  int n_sinks;      // sink slots [0, n_sinks), one per listed sink (-1 where dropped)
   int gen_start;    // first slot of the current block
   int blk_start;    // first slot of the kept blocks
   int pad_bs;       // slots per kept block
@@ -50,17 +51,23 @@ __device__ __forceinline__ LayoutPrefetch layout_prefetch(const int32_t* blk_g, 
   return pf;
 }
 
-__device__ __forceinline__ SlotLayout build_sparse_layout(const LayoutPrefetch& pf, const int32_t* blk_g, int C,
-                                                          const int32_t* snk_g, int S, int L, int P, int bs, int g0,
-                                                          int g1, int gen_pad, int box_rows, const FastDiv& pad_div,
-                                                          const FastDiv& bs_div, int* s_blk, int max_blocks,
-                                                          int* s_sinks, int max_sinks, SlotLayout* out) {
+// The block part of the layout of (b, h), built by one warp from `pf` (layout_prefetch of
+// the same lists): copies the kept-block list to s_blk (up to max_blocks entries; valid
+// entries first, ascending, then -1) and places the segments. The sink segment has a
+// fixed size, n_sinks = min(S, max_sinks) slots rounded up to box_rows, so no slot
+// position depends on which sinks survive de-duplication (dedupe_sinks). gen_pad = slots
+// given to the current block, box_rows = rows per TMA box (a power of two dividing gen_pad
+// and round_up(bs, 8)); pad_div divides by round_up(bs, 8) (exact below n_slots + 128).
+// Lane 0 writes *out; the layout is also returned to every lane of the warp.
+__device__ __forceinline__ SlotLayout build_block_layout(const LayoutPrefetch& pf, const int32_t* blk_g, int C, int S,
+                                                         int P, int bs, int gen_pad, int box_rows,
+                                                         const FastDiv& pad_div, int* s_blk, int max_blocks,
+                                                         int max_sinks, SlotLayout* out) {
   const int lane = threadIdx.x & 31;
-  const int pre_b0 = pf.b0, pre_b1 = pf.b1, pre_s0 = pf.s0;
   int nvb = 0;
   for (int i0 = 0; i0 < C; i0 += 32) {
     const int i = i0 + lane;
-    const int v = i0 == 0 ? pre_b0 : i0 == 32 ? pre_b1 : ((i < C) ? blk_g[i] : -1);
+    const int v = i0 == 0 ? pf.b0 : i0 == 32 ? pf.b1 : ((i < C) ? blk_g[i] : -1);
     const unsigned m = __ballot_sync(0xffffffffu, v >= 0);
     if (v >= 0 && i < max_blocks) s_blk[i] = v;
     nvb += __popc(m);
@@ -68,18 +75,37 @@ __device__ __forceinline__ SlotLayout build_sparse_layout(const LayoutPrefetch& 
   }
   nvb = min(nvb, max_blocks);
   __syncwarp();
-  int last_size = bs;
-  if (nvb > 0) last_size = min(bs, P - s_blk[nvb - 1] * bs);
-  int nf = 0, prev_last = -1;
-  for (int i0 = 0; i0 < S; i0 += 32) {
+  SlotLayout sl;
+  sl.pad_bs = (bs + 7) & ~7;
+  sl.nvb = nvb;
+  sl.last_size = nvb > 0 ? min(bs, P - s_blk[nvb - 1] * bs) : bs;
+  sl.n_sinks = min(S, max_sinks);
+  sl.gen_start = (sl.n_sinks + box_rows - 1) & ~(box_rows - 1);
+  sl.blk_start = sl.gen_start + gen_pad;
+  sl.n_slots = sl.blk_start + nvb * sl.pad_bs;
+  sl.pad_div = pad_div;
+  if (lane == 0) *out = sl;
+  return sl;
+}
+
+// Sink slots of (b, h), by one warp after build_block_layout: s_sinks[i], i < sl.n_sinks,
+// is sink i, or -1 when it is dropped -- out of range, inside the current block [g0, g1),
+// a repeat of the previous entry (the list is ascending among its valid entries) or
+// inside a kept block. bs_div divides by bs (exact below L).
+__device__ __forceinline__ void dedupe_sinks(const LayoutPrefetch& pf, const int32_t* snk_g, const SlotLayout& sl,
+                                             int L, int P, int g0, int g1, const FastDiv& bs_div, const int* s_blk,
+                                             int* s_sinks) {
+  const int lane = threadIdx.x & 31;
+  int prev_last = -1;
+  for (int i0 = 0; i0 < sl.n_sinks; i0 += 32) {
     const int i = i0 + lane;
-    const int j = i0 == 0 ? pre_s0 : ((i < S) ? snk_g[i] : -1);
+    const int j = i0 == 0 ? pf.s0 : ((i < sl.n_sinks) ? snk_g[i] : -1);
     const int jprev = __shfl_up_sync(0xffffffffu, j, 1);
     const int before = (lane == 0) ? prev_last : jprev;
     bool keep = (j >= 0) && (j < L) && !(j >= g0 && j < g1) && (j != before);
     if (keep && j < P) {
       const int jb = static_cast<int>(bs_div.div(static_cast<uint32_t>(j)));
-      int lo = 0, hi = nvb - 1;
+      int lo = 0, hi = sl.nvb - 1;
       while (lo <= hi) {
         const int mid = (lo + hi) >> 1;
         const int v = s_blk[mid];
@@ -91,23 +117,10 @@ __device__ __forceinline__ SlotLayout build_sparse_layout(const LayoutPrefetch& 
         else hi = mid - 1;
       }
     }
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    const int pos = nf + __popc(m & ((1u << lane) - 1u));
-    if (keep && pos < max_sinks) s_sinks[pos] = j;
-    nf += __popc(m);
+    if (i < sl.n_sinks) s_sinks[i] = keep ? j : -1;
     prev_last = __shfl_sync(0xffffffffu, j, 31);
   }
-  SlotLayout sl;
-  sl.pad_bs = (bs + 7) & ~7;
-  sl.nvb = nvb;
-  sl.last_size = last_size;
-  sl.n_fsinks = min(nf, max_sinks);
-  sl.gen_start = (sl.n_fsinks + box_rows - 1) & ~(box_rows - 1);
-  sl.blk_start = sl.gen_start + gen_pad;
-  sl.n_slots = sl.blk_start + nvb * sl.pad_bs;
-  sl.pad_div = pad_div;
-  if (lane == 0) *out = sl;
-  return sl;
+  __syncwarp();
 }
 
 // First key of the contiguous run starting at group slot gs (box-aligned), or -1 when the
@@ -122,16 +135,16 @@ __device__ __forceinline__ int group_key0(const SlotLayout& sl, const int* s_blk
   return s_blk[i] * bs + (rel - i * sl.pad_bs);
 }
 
-// Key of a sink-segment slot, or -1 for sink padding.
+// Key of a sink-segment slot, or -1 for padding and dropped sinks.
 __device__ __forceinline__ int sink_slot_key(const SlotLayout& sl, const int* s_sinks, int slot) {
-  return (slot >= 0 && slot < sl.n_fsinks) ? s_sinks[slot] : -1;
+  return (slot >= 0 && slot < sl.n_sinks) ? s_sinks[slot] : -1;
 }
 
-// Whether a slot holds a key of the set (not padding, not past the end).
+// Whether a slot holds a key of the set (not padding, not a dropped sink, not past the end).
 template <bool SPARSE>
-__device__ __forceinline__ bool slot_valid(const SlotLayout& sl, int L, int bs, int G, int slot) {
+__device__ __forceinline__ bool slot_valid(const SlotLayout& sl, const int* s_sinks, int L, int bs, int G, int slot) {
   if (!SPARSE) return slot < L;
-  if (slot < sl.gen_start) return slot < sl.n_fsinks;
+  if (slot < sl.gen_start) return slot < sl.n_sinks && s_sinks[slot] >= 0;
   if (slot < sl.blk_start) return (slot - sl.gen_start) < G;
   if (slot >= sl.n_slots) return false;
   const int rel = slot - sl.blk_start;
