@@ -13,7 +13,7 @@ later generation positions [g1, L) are still [MASK].
 from __future__ import annotations
 
 import dataclasses
-from typing import Optional
+from typing import Optional, List
 
 
 @dataclasses.dataclass(frozen=True)
@@ -39,6 +39,10 @@ class FocusConfig:
     n_planted_sinks: int   # sink positions planted in the keys (same in every layer)
     positional: bool       # add the seeded rank-8 smooth positional component to Q and K
     seed: int
+    # variants the pages describe (defaults: the configs' plain schedule)
+    dense_tail: int = 0            # the last dense_tail layers also run dense (Dream keeps 4)
+    relevance: str = "active"      # block relevance from "active" (I_active) or "focus" (I_focus) rows
+    sink_agg: str = "probs"        # sink importance: "probs" (sum of softmax rows) or "mean_query"
 
     @property
     def g0(self) -> int:
@@ -72,8 +76,27 @@ class FocusConfig:
         """Upper bound on |I_p| = S + C*bs + G keys (before de-duplication)."""
         return self.S + min(self.C, self.nb) * self.bs + self.G
 
+    @property
+    def dense_layers(self) -> List[int]:
+        """Layers 0..l_dense, then the last dense_tail layers."""
+        tail = range(max(self.l_dense + 1, self.n_layers - self.dense_tail), self.n_layers)
+        return list(range(min(self.l_dense + 1, self.n_layers))) + list(tail)
+
+    @property
+    def sparse_layers(self) -> List[int]:
+        dense = set(self.dense_layers)
+        return [l for l in range(self.n_layers) if l not in dense]
+
     def replace(self, **kw) -> "FocusConfig":
         return dataclasses.replace(self, **kw)
+
+
+def ratio_forms(cfg: FocusConfig, alpha: float = 0.5, sink_frac: float = 0.01) -> FocusConfig:
+    """The pages' ratio forms of C and S (reproducibility section: alpha = 0.5,
+    N_sinks = 0.01 x M): C = ceil(alpha * nb) kept prompt blocks and S = ceil(sink_frac * L)
+    sinks, L (the context length) standing for M."""
+    import math
+    return cfg.replace(C=max(1, math.ceil(alpha * cfg.nb)), S=max(1, math.ceil(sink_frac * cfg.L)))
 
 
 TINY = FocusConfig(

@@ -5,6 +5,8 @@
 // R_b of the active queries to each block keeps the top-C blocks. Reading fixed by the
 // build's specification: R_b^h = mean over the active queries and the query heads of
 // KV group h of q . kbar_b / sqrt(d), which equals qbar_h . kbar_b / sqrt(d).
+#include <algorithm>
+
 #include "focus_common.cuh"
 #include "topk.cuh"
 
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   griddep_wait();               // inputs may come from the previous kernel on the stream
   griddep_launch_dependents();
   constexpr int PARTS = kSelectThreads / D;
-  extern __shared__ float s_R[];           // [nb], gathered in CTA 0
+  extern __shared__ float s_R[];           // [nb] gathered in CTA 0, then [2048 + 64] top-C histogram
   __shared__ float s_part[PARTS][D];
   __shared__ float s_qbar[D];
   __shared__ TopkShared tk;
@@ -145,9 +147,10 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   if (rank != 0) return;
   int32_t* out = blocks + static_cast<size_t>(bh) * C;
   auto key_of = [&](int i) { return float_order_key(s_R[i]); };
-  if (nb <= kSelectThreads) block_topk_small<1>(key_of, nb, C, out, C, tk);
-  else if (nb <= 2 * kSelectThreads) block_topk_small<2>(key_of, nb, C, out, C, tk);
-  else if (nb <= 4 * kSelectThreads) block_topk_small<4>(key_of, nb, C, out, C, tk);
+  int* wide = reinterpret_cast<int*>(s_R + ((nb + 3) & ~3));
+  if (nb <= kSelectThreads) block_topk_small<1>(key_of, nb, C, out, C, tk, wide);
+  else if (nb <= 2 * kSelectThreads) block_topk_small<2>(key_of, nb, C, out, C, tk, wide);
+  else if (nb <= 4 * kSelectThreads) block_topk_small<4>(key_of, nb, C, out, C, tk, wide);
   else block_topk_ascending(key_of, nb, C, out, C, tk);
 }
 
@@ -192,12 +195,12 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
     set_error("head dim %d unsupported (64 or 128)", d);
     return FOCUS_ERR_UNSUPPORTED;
   }
-  if (nb > 16384) {
-    set_error("nb=%d exceeds 16384 blocks", nb);
+  if (nb > 49152) {
+    set_error("nb=%d exceeds 49152 blocks", nb);
     return FOCUS_ERR_UNSUPPORTED;
   }
   if (B == 0) return FOCUS_OK;
-  const size_t smem = static_cast<size_t>(nb) * sizeof(float);
+  const size_t smem = (static_cast<size_t>((nb + 3) & ~3) + 2048 + 64) * sizeof(float);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const __nv_bfloat16* q = reinterpret_cast<const __nv_bfloat16*>(Q_active);
   // cluster of cs CTAs per (sequence, KV head), cs a power of two with B*Hkv*cs <= SMs
@@ -208,18 +211,20 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
   while (cs < 8 && units * cs * 2 <= device_sm_count() && (nb + cs * 2 - 1) / (cs * 2) >= 16) cs *= 2;
   cudaError_t err;
   if (d == 128) {
-    static bool cfg = false;
-    if (!cfg) {
-      cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
-      cfg = true;
+    static size_t cfg = 0;             // dynamic shared memory the kernel is configured for
+    if (smem > cfg) {
+      cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(std::max<size_t>(smem, 80 * 1024)));
+      cfg = std::max<size_t>(smem, 80 * 1024);
     }
     err = launch_k_cluster(block_select_kernel<128>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
                            n_active, kbar, Hq, Hkv, acap, acap_div, nb, C, blocks, scores_opt);
   } else {
-    static bool cfg = false;
-    if (!cfg) {
-      cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
-      cfg = true;
+    static size_t cfg = 0;
+    if (smem > cfg) {
+      cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(std::max<size_t>(smem, 80 * 1024)));
+      cfg = std::max<size_t>(smem, 80 * 1024);
     }
     err = launch_k_cluster(block_select_kernel<64>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
                            n_active, kbar, Hq, Hkv, acap, acap_div, nb, C, blocks, scores_opt);

@@ -354,8 +354,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (cs > 1) cluster_sync();   // every CTA holds all nb keys
     else __syncthreads();
     auto key_of = [&](int i) { return s_key[i]; };
-    if (a.nb <= 4 * kDecThreads) block_topk_small<4>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
-    else if (a.nb <= 8 * kDecThreads) block_topk_small<8>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
+    int* s_wide = reinterpret_cast<int*>(sK + 4096);          // 11-bit first-pass histogram
+    static_assert((RG + 1) * D * 4 <= 4096, "qbar partials overlap the top-C histogram");
+    if (a.nb <= 4 * kDecThreads) block_topk_small<4>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk, s_wide);
+    else if (a.nb <= 8 * kDecThreads) block_topk_small<8>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk, s_wide);
     else block_topk_ascending(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
     __syncthreads();
     if (rank == 0 && a.blocks_out)

@@ -90,6 +90,29 @@ __global__ void gather_rows_kernel(const uint4* __restrict__ X, const int32_t* _
   out[idx] = v;
 }
 
+// Inverse of gather_rows: one thread per 16-byte chunk of a (matrix, b, h, listed row).
+__global__ void scatter_rows_kernel(uint4* __restrict__ X, const int32_t* __restrict__ rows,
+                                    const int32_t* __restrict__ n_rows, int B, int H, int L, int chunks, int cap,
+                                    long long total, const uint4* __restrict__ src_rows, int* dev_err) {
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int c = static_cast<int>(idx % chunks);
+  long long r = idx / chunks;
+  const int i = static_cast<int>(r % cap);
+  r /= cap;
+  const long long mbh = r;                 // (m * B + b) * H + h
+  const int b = static_cast<int>((mbh / H) % B);
+  if (i >= n_rows[b]) return;
+  const int dst = rows[static_cast<size_t>(b) * cap + i];
+  if (dst < 0 || dst >= L) {
+    record_dev_error(dev_err, DEV_ERR_BAD_INDEX);
+    return;
+  }
+  X[(mbh * L + dst) * chunks + c] = __ldg(src_rows + idx);
+}
+
 }  // namespace focus
 
 using namespace focus;
@@ -150,6 +173,30 @@ extern "C" int focus_gather_rows(const focus_bf16* X, const int32_t* rows, const
   note_launch();
   if (e != cudaSuccess) {
     set_error("gather_rows launch: %s", cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
+}
+
+extern "C" int focus_scatter_rows(focus_bf16* X, const int32_t* rows, const int32_t* n_rows, int n_mat, int B, int H,
+                                  int L, int d, int cap, const focus_bf16* X_rows, void* stream) {
+  FOCUS_CHECK_ARG(X && rows && n_rows && X_rows, "null pointer argument");
+  FOCUS_CHECK_ARG(n_mat >= 0 && B >= 0 && H >= 1 && L >= 1 && cap >= 1, "bad sizes");
+  FOCUS_CHECK_ARG(d % 8 == 0 && d > 0, "d must be a positive multiple of 8");
+  FOCUS_CHECK_ARG(aligned16(X) && aligned16(X_rows), "tensors must be 16-byte aligned");
+  const int chunks = d / 8;
+  const long long total = static_cast<long long>(n_mat) * B * H * cap * chunks;
+  if (total == 0) return FOCUS_OK;
+  const int threads = 256;
+  const long long blocks = (total + threads - 1) / threads;
+  FOCUS_CHECK_ARG(blocks < (1LL << 31), "too large");
+  const cudaError_t e =
+      launch_k(scatter_rows_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+               static_cast<cudaStream_t>(stream), reinterpret_cast<uint4*>(X), rows, n_rows, B, H, L, chunks, cap,
+               total, reinterpret_cast<const uint4*>(X_rows), device_error_word());
+  note_launch();
+  if (e != cudaSuccess) {
+    set_error("scatter_rows launch: %s", cudaGetErrorString(e));
     return FOCUS_ERR_CUDA;
   }
   return FOCUS_OK;

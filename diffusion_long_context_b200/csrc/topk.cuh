@@ -185,9 +185,12 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
 // priv (optional): 2 * (blockDim.x / 32) * 257 ints of shared memory for per-warp
 // histograms (padded so that the warps' copies of a bin sit in different banks); with it
 // a bin holding most of the keys costs no cross-warp atomic serialisation.
+// wide (optional): 2048 + 64 ints of shared memory. With it the first pass takes 11 bits
+// (a 2048-bin histogram and its 64-bin coarse sums, searched coarse then fine), which for
+// a few hundred smooth keys almost always isolates the k-th key in one pass.
 template <int KPT>
 __device__ void block_topk_small_regs(uint32_t (&key)[KPT], int n, int k, int32_t* out, int cap,
-                                      TopkShared& sm, int* priv = nullptr) {
+                                      TopkShared& sm, int* priv = nullptr, int* wide = nullptr) {
   const int tid = threadIdx.x, nt = blockDim.x;
   const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
   k = min(k, n);
@@ -216,6 +219,8 @@ __device__ void block_topk_small_regs(uint32_t (&key)[KPT], int n, int k, int32_
   for (int i = tid; i < 256; i += nt) sm.hist[i] = 0;
   if (priv)
     for (int i = tid; i < nwarps * 257; i += nt) priv[i] = 0;
+  if (wide)
+    for (int i = tid; i < 2048 + 64; i += nt) wide[i] = 0;
   __syncthreads();
   for (int w = 0; w < nwarps; ++w) {
     kmin = min(kmin, static_cast<uint32_t>(sm.w_gt[w]));
@@ -230,6 +235,45 @@ __device__ void block_topk_small_regs(uint32_t (&key)[KPT], int n, int k, int32_
   int remaining = k;
   int buf = 0;
   bool whole = (range == 0u);          // all keys equal: take the lowest indices
+  auto warp_incl_scan = [&](int v) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    return v;
+  };
+  if (wide && hi >= 11 && !whole) {
+    int* fine = wide;
+    int* coarse = wide + 2048;
+    const int lo = hi - 11;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      if (tid * KPT + j < n) {
+        const uint32_t f = (key[j] >> lo) & 2047u;
+        atomicAdd(&fine[f], 1);
+        atomicAdd(&coarse[f >> 5], 1);
+      }
+    }
+    __syncthreads();
+    // coarse digit: lane l owns coarse bins 63-2l, 62-2l (descending)
+    const int ca = coarse[63 - 2 * lane], cb = coarse[62 - 2 * lane];
+    const int incl = warp_incl_scan(ca + cb);
+    const int excl = incl - (ca + cb);
+    const int L = __ffs(__ballot_sync(0xffffffffu, incl >= remaining)) - 1;
+    const bool first = excl + ca >= remaining;
+    const int cd = __shfl_sync(0xffffffffu, first ? 63 - 2 * lane : 62 - 2 * lane, L);
+    remaining -= __shfl_sync(0xffffffffu, first ? excl : excl + ca, L);
+    // fine digit inside coarse bin cd: lane l owns fine bin cd*32 + 31 - l
+    const int cf = fine[cd * 32 + 31 - lane];
+    const int incl2 = warp_incl_scan(cf);
+    const int L2 = __ffs(__ballot_sync(0xffffffffu, incl2 >= remaining)) - 1;
+    const int cnt = __shfl_sync(0xffffffffu, cf, L2);
+    remaining -= __shfl_sync(0xffffffffu, incl2 - cf, L2);
+    whole = (cnt == remaining);
+    P = static_cast<uint32_t>(cd * 32 + 31 - L2);
+    hi = lo;
+  }
   while (hi > 0 && !whole) {
     const int lo = max(0, hi - 8);
     int* hist = buf ? sm.hist2 : sm.hist;
@@ -340,14 +384,15 @@ __device__ void block_topk_small_regs(uint32_t (&key)[KPT], int n, int k, int32_
 }
 
 template <int KPT, typename KeyFn>
-__device__ void block_topk_small(KeyFn key_of, int n, int k, int32_t* out, int cap, TopkShared& sm) {
+__device__ void block_topk_small(KeyFn key_of, int n, int k, int32_t* out, int cap, TopkShared& sm,
+                                 int* wide = nullptr) {
   uint32_t key[KPT];
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
     const int i = threadIdx.x * KPT + j;
     key[j] = i < n ? key_of(i) : 0u;
   }
-  block_topk_small_regs<KPT>(key, n, k, out, cap, sm);
+  block_topk_small_regs<KPT>(key, n, k, out, cap, sm, nullptr, wide);
 }
 
 }  // namespace focus

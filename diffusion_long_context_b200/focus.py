@@ -37,6 +37,7 @@ _SIGS = {
     "focus_device_error": (_i, [ctypes.POINTER(ctypes.c_int)]),
     "focus_select_queries": (_i, [_p, _p, _i, _i, _i, _i, _i, _f, _i, _p, _p, _i, _p, _p, _i, _p]),
     "focus_gather_rows": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]),
+    "focus_scatter_rows": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]),
     "focus_block_means": (_i, [_p, _i, _i, _i, _i, _i, _i, _p, _p]),
     "focus_block_select": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "focus_dense_attention": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
@@ -131,6 +132,22 @@ def focus_gather_rows(X, rows, n_rows, X_rows, stream=None):
     st = lib.focus_gather_rows(_ptr(X), _ptr(rows), _ptr(n_rows), n_mat, B, H, L, d, cap, _ptr(X_rows),
                                _stream(stream))
     _check(st, "focus_gather_rows")
+
+
+def focus_scatter_rows(X, rows, n_rows, X_rows, stream=None):
+    """Approximate-KV-cache refresh: X[..., rows[b, i], :] = X_rows[..., i, :] for i < n_rows[b].
+
+    X [n_mat, B, H, L, d] (or [B, H, L, d]) is updated in place from X_rows [..., cap, d]."""
+    _need(X, torch.bfloat16, "X")
+    _need(X_rows, torch.bfloat16, "X_rows")
+    _need(rows, torch.int32, "rows", 2)
+    _need(n_rows, torch.int32, "n_rows", 1)
+    x = X if X.dim() == 5 else X.unsqueeze(0)
+    n_mat, B, H, L, d = x.shape
+    cap = rows.shape[1]
+    st = lib.focus_scatter_rows(_ptr(X), _ptr(rows), _ptr(n_rows), n_mat, B, H, L, d, cap, _ptr(X_rows),
+                                _stream(stream))
+    _check(st, "focus_scatter_rows")
 
 
 def focus_block_means(K, P, bs, kbar, stream=None):

@@ -29,7 +29,9 @@ class SparseStep:
         """Q_full [n_layers, B, Hq, L, d]; K[l], V[l] [B, Hkv, L, d] (bf16, on `device`).
 
         fused: each sparse layer runs block relevance + top-C and the sparse attention as
-        one launch (focus_sparse_attention_fused), else as two calls."""
+        one launch (focus_sparse_attention_fused), else as two calls. The config's variants
+        (dense_tail, relevance, sink_agg) change the schedule; relevance="focus" runs the
+        two calls."""
         c = cfg
         self.cfg = c
         self.fused = fused
@@ -50,7 +52,17 @@ class SparseStep:
         self.O_active = torch.zeros((c.n_layers, c.B, c.Hq, c.acap, c.d), **bf)
         self.colsum = torch.zeros((c.B, c.Hkv, c.L), dtype=torch.float32, device=self.dev)
         self.sinks = torch.full((c.B, c.Hkv, c.S), -1, **i32)
-        self.sparse_layers = list(range(c.l_dense + 1, c.n_layers))
+        self.dense_layers = c.dense_layers
+        self.sparse_layers = c.sparse_layers
+        # variants: relevance from the I_focus rows needs their queries (and the two-call
+        # layer, the fused kernel scores with the rows it attends with); mean-query sinks
+        # score every key of the sink layer, held as fp32 "blocks" of one key
+        self.Q_focus = (torch.zeros((c.n_layers, c.B, c.Hq, self.kcap, c.d), **bf) if c.relevance == "focus"
+                        else None)
+        if c.relevance == "focus":
+            self.fused = False
+        self.k_rows = (torch.zeros((c.B, c.Hkv, c.L, c.d), dtype=torch.float32, device=self.dev)
+                       if c.sink_agg == "mean_query" else None)
         self.kbar = {l: torch.zeros((c.B, c.Hkv, c.nb, c.d), dtype=torch.float32, device=self.dev)
                      for l in self.sparse_layers}
         self.blocks = {l: torch.full((c.B, c.Hkv, c.C), -1, **i32) for l in self.sparse_layers}
@@ -82,17 +94,27 @@ class SparseStep:
         F.focus_select_queries(self.conf_prev, self.mask, c.g0, c.g1, c.n_t, self.rho, c.w, self.i_focus,
                                self.n_focus, self.i_active, self.n_active)
         F.focus_gather_rows(self.Q_full, self.i_active, self.n_active, self.Q_active)
+        if self.Q_focus is not None:
+            F.focus_gather_rows(self.Q_full, self.i_focus, self.n_focus, self.Q_focus)
 
     def dense_layer(self, l: int):
         c = self.cfg
-        want = l == c.l_dense
+        sink_layer = l == c.l_dense
+        probs = sink_layer and c.sink_agg == "probs"
         F.focus_dense_attention(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.O_active[l],
-                                scale=self.scale, colsum=self.colsum if want else None, ws=self.ws)
-        if want:
+                                scale=self.scale, colsum=self.colsum if probs else None, ws=self.ws)
+        if probs:
             F.focus_sink_identify(self.colsum, c.S, self.sinks)
+        elif sink_layer:
+            # mean-query importance: top-S of qbar . k_j over all L keys (each key a block of one)
+            F.focus_block_means(self.K[l], c.L, 1, self.k_rows)
+            F.focus_block_select(self.Q_active[l], self.n_active, self.k_rows, c.S, self.sinks)
 
     def block_select_layer(self, l: int):
-        F.focus_block_select(self.Q_active[l], self.n_active, self.kbar[l], self.cfg.C, self.blocks[l])
+        if self.Q_focus is not None:
+            F.focus_block_select(self.Q_focus[l], self.n_focus, self.kbar[l], self.cfg.C, self.blocks[l])
+        else:
+            F.focus_block_select(self.Q_active[l], self.n_active, self.kbar[l], self.cfg.C, self.blocks[l])
 
     def sparse_attention_layer(self, l: int):
         c = self.cfg
@@ -122,10 +144,11 @@ class SparseStep:
             timers.setdefault(kind, []).append((s, e))
 
         timed("select", self.select)
-        for l in range(min(c.l_dense + 1, c.n_layers)):
-            timed("dense_attention" if l != c.l_dense else "dense_attention_colsum", self.dense_layer, l)
-        for l in self.sparse_layers:
-            if self.fused:
+        dense = set(self.dense_layers)
+        for l in range(c.n_layers):
+            if l in dense:
+                timed("dense_attention" if l != c.l_dense else "dense_attention_colsum", self.dense_layer, l)
+            elif self.fused:
                 timed("sparse_layer_fused", self.sparse_layer_fused, l)
             else:
                 timed("block_select", self.block_select_layer, l)

@@ -105,6 +105,21 @@ FOCUS_API int focus_gather_rows(const focus_bf16* X, const int32_t* rows, const 
                       int L, int d, int cap, focus_bf16* X_rows, void* stream);
 
 /*
+ * Approximate-KV-cache refresh (Focus-dLLM summary page, "近似KV缓存" / approximate KV
+ * cache: a token of the refresh set U(t) takes its recomputed key and value, every other
+ * token keeps its cached one). The inverse of focus_gather_rows: for every matrix m,
+ * X[m, b, h, rows[b, i]] = X_rows[m, b, h, i] for i < n_rows[b]; all other rows of X are
+ * left unchanged. X [n_mat, B, H, L, d] (the K or V cache of n_mat layers, updated in
+ * place), X_rows [n_mat, B, H, cap, d], rows [B, cap] and n_rows [B] int32 (device), e.g.
+ * I_active (or I_focus) from focus_select_queries. Row lists must not repeat a row (the
+ * selection outputs are ascending and unique). Indices outside [0, L) are skipped and
+ * flagged in the device error word (code 5). d a multiple of 8; X and X_rows 16-byte
+ * aligned. The pages have no fused form of this step; it runs as one scatter launch.
+ */
+FOCUS_API int focus_scatter_rows(focus_bf16* X, const int32_t* rows, const int32_t* n_rows, int n_mat, int B, int H,
+                                 int L, int d, int cap, const focus_bf16* X_rows, void* stream);
+
+/*
  * (4a) Block representative keys -- method steps (4): the prompt [0, P) is cut into
  * nb = ceil(P / bs) contiguous blocks; kbar[b, h, j] = mean of K[b, h, j*bs : min(P,(j+1)*bs)].
  * K [B, Hkv, L, d] bf16 -> kbar [B, Hkv, nb, d] fp32. Requires 1 <= P <= L, bs >= 1,
@@ -119,7 +134,7 @@ FOCUS_API int focus_block_means(const focus_bf16* K, int B, int Hkv, int L, int 
  * KV group h of q . kbar[b, h, j] / sqrt(d) (0 when n_active[b] == 0).
  * blocks[b, h, :] = the top-min(C, nb) blocks, ascending, -1 tail.
  * Q_active [B, Hq, acap, d] bf16; n_active [B]; kbar [B, Hkv, nb, d] fp32;
- * scores_opt: NULL or [B, Hkv, nb] fp32 receiving R. Requires nb <= 16384, C >= 1,
+ * scores_opt: NULL or [B, Hkv, nb] fp32 receiving R. Requires nb <= 49152, C >= 1,
  * d in {64, 128}.
  */
 FOCUS_API int focus_block_select(const focus_bf16* Q_active, const int32_t* n_active, const float* kbar, int B, int Hq,

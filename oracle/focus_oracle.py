@@ -103,6 +103,18 @@ def gather_rows(X: np.ndarray, rows: Sequence[np.ndarray], cap: int) -> np.ndarr
 
 
 # --------------------------------------------------------- step (4): block means
+def refresh_rows(X: np.ndarray, rows: Sequence[np.ndarray], X_new: np.ndarray) -> np.ndarray:
+    """Approximate KV cache (summary page, "近似KV缓存"): a token i of the refresh set U(t)
+    takes its recomputed state, every other token keeps the cached one:
+    X'[b, h, i] = X_new[b, h, k] where rows[b][k] == i, else X[b, h, i].
+    X [B, H, L, d], X_new [B, H, cap, d] (row k of sequence b for k < len(rows[b]))."""
+    out = X.copy()
+    for b, r in enumerate(rows):
+        for k, i in enumerate(r):
+            out[b, :, int(i)] = X_new[b, :, k]
+    return out
+
+
 def block_means(K: np.ndarray, P: int, bs: int) -> np.ndarray:
     """Representative key of each prompt block = mean of the block's keys.
 
@@ -254,10 +266,21 @@ def sparse_attention(Q_active: np.ndarray, n_active: Sequence[int], K: np.ndarra
 
 
 # ------------------------------------------------------------- the step schedule
+def sink_identify_mean_query(Q_active: np.ndarray, n_active: Sequence[int], K: np.ndarray,
+                             S: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Variant sink importance (summary page, "方法步骤详情" (3): token importance from an
+    aggregated query representation): the attention of the group's mean active query,
+    softmax_j(qbar . k_j / sqrt(d)), over all L columns. The softmax is monotone in the
+    score, so the top-S columns are the top-S of R_j = qbar . k_j / sqrt(d): block relevance
+    with every key its own block. Returns (sinks [B,Hkv,S], R)."""
+    return block_select(Q_active, n_active, K, S)
+
+
 def sparse_step(layer_fn: Callable[[int], Tuple[np.ndarray, np.ndarray, np.ndarray]],
                 n_layers: int, l_dense: int, conf_prev: np.ndarray, mask: np.ndarray,
                 g0: int, g1: int, n_t: int, rho: float, w: int, P: int, bs: int,
-                C: int, S: int, acap: int, scale: float, layers_out=None):
+                C: int, S: int, acap: int, scale: float, layers_out=None, dense_tail: int = 0,
+                relevance: str = "active", sink_agg: str = "probs"):
     """One non-block-entry denoising step (method steps (1)-(5)).
 
     layer_fn(l) -> (Q_full [B,Hq,L,d], K, V) in float64. Layers 0..l_dense are dense over
@@ -265,22 +288,37 @@ def sparse_step(layer_fn: Callable[[int], Tuple[np.ndarray, np.ndarray, np.ndarr
     blocks from their own block means and attend over sinks U blocks U the current block.
     Returns a dict with I_focus, I_active, sinks, per-layer blocks and outputs (only for
     layers in `layers_out`, default all).
+
+    Variants the pages describe: the last `dense_tail` layers also run dense (Dream keeps
+    its last 4 layers dense); relevance="focus" scores the blocks with the I_focus rows
+    instead of I_active (method steps (4) speaks of the candidate queries);
+    sink_agg="mean_query" picks the sinks by the mean active query's attention
+    (sink_identify_mean_query) instead of the summed softmax rows.
     """
     focus, active = select_queries(conf_prev, mask, g0, g1, n_t, rho, w)
     n_active = [a.size for a in active]
     out = {"I_focus": focus, "I_active": active, "O": {}, "blocks": {}, "sinks": None}
     want = set(range(n_layers)) if layers_out is None else set(layers_out)
+    tail0 = max(l_dense + 1, n_layers - dense_tail)
     for l in range(n_layers):
         Q, K, V = layer_fn(l)
         Qa = gather_rows(Q, active, acap)
-        if l <= l_dense:
-            O, colsum, _ = dense_attention(Qa, n_active, K, V, scale, want_colsum=(l == l_dense))
-            if l == l_dense:
-                out["sinks"] = sink_identify(colsum, S)
-                out["colsum"] = colsum
+        if l <= l_dense or l >= tail0:
+            sink_layer = l == l_dense
+            O, colsum, _ = dense_attention(Qa, n_active, K, V, scale, want_colsum=sink_layer and sink_agg == "probs")
+            if sink_layer:
+                if sink_agg == "probs":
+                    out["sinks"] = sink_identify(colsum, S)
+                    out["colsum"] = colsum
+                else:
+                    out["sinks"], out["sink_scores"] = sink_identify_mean_query(Qa, n_active, K, S)
         else:
             kbar = block_means(K, P, bs)
-            blocks, _ = block_select(Qa, n_active, kbar, C)
+            if relevance == "focus":
+                Qr = gather_rows(Q, focus, g1 - g0)
+                blocks, _ = block_select(Qr, [f.size for f in focus], kbar, C)
+            else:
+                blocks, _ = block_select(Qa, n_active, kbar, C)
             out["blocks"][l] = blocks
             O = sparse_attention(Qa, n_active, K, V, out["sinks"], blocks, bs, P, g0, g1, scale)
         if l in want:

@@ -109,6 +109,38 @@ def test_gather_rows(F):
     assert F.device_error() == 0
 
 
+# ------------------------------------------------------------------ KV-cache refresh
+def test_scatter_rows_matches_oracle_refresh(F):
+    """Approximate-KV-cache refresh over a stack of layers: bit-exact against the oracle."""
+    X = inputs.random_bf16((3, 2, 5, 300, 128), seed=8, device=DEV)
+    Xn = inputs.random_bf16((3, 2, 5, 6, 128), seed=9, device=DEV)
+    rows = torch.tensor([[0, 7, 8, 299, -1, -1], [1, 2, 3, 4, 5, 6]], dtype=torch.int32, device=DEV)
+    n = torch.tensor([4, 6], dtype=torch.int32, device=DEV)
+    ref_in = X.cpu()
+    F.focus_scatter_rows(X, rows, n, Xn)
+    torch.cuda.synchronize()
+    rl = [rows[0, :4].cpu().numpy(), rows[1, :6].cpu().numpy()]
+    for m in range(3):
+        want = orc.refresh_rows(ref_in[m].float().numpy(), rl, Xn[m].cpu().float().numpy())
+        assert np.array_equal(X[m].cpu().float().numpy(), want)
+    assert F.device_error() == 0
+
+
+def test_scatter_rows_empty_and_out_of_range(F):
+    X = inputs.random_bf16((2, 2, 40, 64), seed=10, device=DEV)
+    before = X.clone()
+    Xn = inputs.random_bf16((2, 2, 4, 64), seed=11, device=DEV)
+    rows = torch.tensor([[3, 5, -1, -1], [40, 1, -1, -1]], dtype=torch.int32, device=DEV)
+    F.focus_scatter_rows(X, rows, torch.tensor([0, 0], dtype=torch.int32, device=DEV), Xn)
+    torch.cuda.synchronize()
+    assert torch.equal(X, before)                                   # empty refresh sets
+    F.focus_scatter_rows(X, rows, torch.tensor([2, 2], dtype=torch.int32, device=DEV), Xn)
+    torch.cuda.synchronize()
+    assert F.device_error() != 0                                    # row 40 is outside [0, 40)
+    assert torch.equal(X[1, :, 1], Xn[1, :, 1]) and torch.equal(X[0, :, 3], Xn[0, :, 0])
+    assert torch.equal(X[1, :, 2:], before[1, :, 2:]) and torch.equal(X[0, :, :3], before[0, :, :3])
+
+
 # ------------------------------------------------------------------ block means
 @pytest.mark.parametrize("d,P,bs,L", [(64, 448, 32, 512), (128, 1000, 64, 1100), (128, 333, 128, 400),
                                       (128, 64, 1, 64), (64, 250, 24, 260)])
@@ -416,4 +448,39 @@ def test_sparse_fused_matches_oracle_and_two_calls(F, case):
                                float(np.float32(1 / math.sqrt(d))))
     assert_attention_close(O_f, ref, rows_valid=n_act, what=f"fused sparse ({name})")
     assert (O_f.float() - O_2.float()).abs().max().item() <= 1e-2
+    assert F.device_error() == 0
+
+
+# ------------------------------------------------------------------ the step sequencer, plain and variants
+@pytest.mark.parametrize("variant", ["plain_fused", "dream_tail_focus_meanq_ratio"])
+def test_sparse_step_sequencer(F, variant):
+    """SparseStep (the product's step schedule) against the oracle's composed step."""
+    from diffusion_long_context_b200 import configs as cf
+    from diffusion_long_context_b200.step import SparseStep
+    cfg = cf.scaled(cf.LLADA_8K, 1024, n_layers=6, Hq=4, Hkv=2, l_dense=1, C=4, S=8)
+    fused = True
+    if variant != "plain_fused":
+        cfg = cf.ratio_forms(cfg.replace(dense_tail=2, relevance="focus", sink_agg="mean_query"))
+        fused = False
+    st = inputs.step_state(cfg)
+    layers = [inputs.make_layer(cfg, l, DEV, st.sink_pos) for l in range(cfg.n_layers)]
+    Q_full = torch.stack([lay[0] for lay in layers])
+    step = SparseStep(cfg, Q_full, [lay[1] for lay in layers], [lay[2] for lay in layers], device=DEV, fused=fused)
+    step.set_state(torch.from_numpy(st.conf_prev), torch.from_numpy(st.mask), non_blocking=False)
+    step.block_entry()
+    step.run()
+    torch.cuda.synchronize()
+    f64 = [tuple(inputs.to_f64(t) for t in lay) for lay in layers]
+    ref = orc.sparse_step(lambda l: f64[l], cfg.n_layers, cfg.l_dense, st.conf_prev, st.mask, cfg.g0, cfg.g1,
+                          cfg.n_t, step.rho, cfg.w, cfg.P, cfg.bs, cfg.C, cfg.S, cfg.acap,
+                          float(np.float32(1 / math.sqrt(cfg.d))), dense_tail=cfg.dense_tail,
+                          relevance=cfg.relevance, sink_agg=cfg.sink_agg)
+    assert idx_rows(step.i_active) == [a.tolist() for a in ref["I_active"]]
+    assert np.array_equal(step.sinks.cpu().numpy(), ref["sinks"]), "sink sets differ"
+    nA = [len(a) for a in ref["I_active"]]
+    assert sorted(ref["blocks"]) == step.sparse_layers
+    for l in range(cfg.n_layers):
+        if l in step.sparse_layers:
+            assert np.array_equal(step.blocks[l].cpu().numpy(), ref["blocks"][l]), f"layer {l} blocks differ"
+        assert_attention_close(step.O_active[l], ref["O"][l], rows_valid=nA, what=f"{variant} layer {l}")
     assert F.device_error() == 0

@@ -350,3 +350,65 @@ def test_sparse_partial_last_block():
     """P % bs != 0: the last block covers only the valid prompt rows [16, 20), not [16, 24)."""
     Ip = orc.sparse_key_set(np.array([-1]), np.array([2]), 8, 20, 28, 32)
     assert Ip.tolist() == [16, 17, 18, 19, 28, 29, 30, 31]
+
+
+# ------------------------------------------------------------------ approximate KV-cache refresh
+def test_refresh_rows_golden_and_invariants():
+    """Summary page, "近似KV缓存": tokens of U(t) take the recomputed state, all others keep
+    the cache. Hand-worked case, then the gather/refresh round trip on random data."""
+    X = np.arange(2 * 1 * 4 * 2, dtype=np.float64).reshape(2, 1, 4, 2)
+    Xn = -np.ones((2, 1, 3, 2))
+    Xn[0, 0, 1] = [-5.0, -6.0]
+    out = orc.refresh_rows(X, [np.array([1, 3]), np.array([], dtype=np.int64)], Xn)
+    want = X.copy()
+    want[0, 0, 1] = [-1.0, -1.0]
+    want[0, 0, 3] = [-5.0, -6.0]
+    assert np.array_equal(out, want)
+    assert np.array_equal(X, np.arange(16, dtype=np.float64).reshape(2, 1, 4, 2))   # input untouched
+    rng = np.random.default_rng(3)
+    Xr = rng.standard_normal((3, 2, 50, 8))
+    rows = [np.sort(rng.choice(50, size=n, replace=False)) for n in (0, 7, 50)]
+    Xnew = rng.standard_normal((3, 2, 50, 8))
+    out = orc.refresh_rows(Xr, rows, Xnew)
+    back = orc.gather_rows(out, rows, 50)
+    for b, r in enumerate(rows):
+        assert np.array_equal(back[b, :, :r.size], Xnew[b, :, :r.size])
+        keep = np.setdiff1d(np.arange(50), r)
+        assert np.array_equal(out[b, :, keep], Xr[b, :, keep])
+
+
+# ------------------------------------------------------------------ step variants
+def test_mean_query_sinks_against_explicit_softmax():
+    """Variant sink importance: the top-S columns of the mean active query's attention row,
+    computed here by an explicit fp64 softmax and a full sort, with a planted key."""
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, A, L, d, S = 2, 4, 2, 5, 200, 16, 6
+    Q = rng.standard_normal((B, Hq, 8, d))
+    K = rng.standard_normal((B, Hkv, L, d))
+    n_active = [5, 3]
+    qbar = np.zeros((B, Hkv, d))
+    for b in range(B):
+        for h in range(Hkv):
+            rows = Q[b, h * 2:(h + 1) * 2, :n_active[b]].reshape(-1, d)
+            qbar[b, h] = rows.mean(axis=0)
+    K[1, 0, 77] = 5.0 * qbar[1, 0] / np.linalg.norm(qbar[1, 0])      # planted: aligned with qbar
+    sinks, _ = orc.sink_identify_mean_query(Q, n_active, K, S)
+    for b in range(B):
+        for h in range(Hkv):
+            s = K[b, h] @ qbar[b, h] / np.sqrt(d)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            order = sorted(range(L), key=lambda j: (-p[j], j))[:S]
+            assert sinks[b, h].tolist() == sorted(order)
+    assert 77 in sinks[1, 0].tolist()
+
+
+def test_variant_schedules_and_ratio_forms():
+    from diffusion_long_context_b200 import configs as cf
+    dream = cf.DREAM_16K.replace(dense_tail=4)
+    assert dream.dense_layers == [0, 1, 2, 24, 25, 26, 27]
+    assert dream.sparse_layers == list(range(3, 24))
+    assert cf.FULL_32K.dense_layers == [0, 1, 2] and cf.FULL_32K.sparse_layers == list(range(3, 32))
+    r = cf.ratio_forms(cf.FULL_32K)               # alpha = 0.5 of 508 blocks, 1% of 32768 tokens
+    assert (r.C, r.S) == (254, 328)
+    assert cf.ratio_forms(cf.TINY).C == 7 and cf.ratio_forms(cf.TINY).S == 6
