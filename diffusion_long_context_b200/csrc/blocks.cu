@@ -148,8 +148,7 @@ __global__ void __launch_bounds__(kSelectThreads) block_select_kernel(
   int32_t* out = blocks + static_cast<size_t>(bh) * C;
   auto key_of = [&](int i) { return float_order_key(s_R[i]); };
   int* wide = reinterpret_cast<int*>(s_R + ((nb + 3) & ~3));
-  if (nb <= kSelectThreads) block_topk_small<1>(key_of, nb, C, out, C, tk, wide);
-  else if (nb <= 2 * kSelectThreads) block_topk_small<2>(key_of, nb, C, out, C, tk, wide);
+  if (nb <= 2 * kSelectThreads) cta_topk_linear<true>(reinterpret_cast<const uint32_t*>(s_R), nb, C, out, C, wide, tk);
   else if (nb <= 4 * kSelectThreads) block_topk_small<4>(key_of, nb, C, out, C, tk, wide);
   else block_topk_ascending(key_of, nb, C, out, C, tk);
 }

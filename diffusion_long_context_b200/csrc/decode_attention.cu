@@ -182,17 +182,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       else tma_load_3d_hint(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh, l2_stream);
     }
     if (SPARSE && tma_mask != all_groups) {
-      // sink rows (and rows past the end, zero-filled) by cp.async, 16 bytes per lane
+      // Sink rows (and rows past the end) by cp.async, 16 bytes per lane: lane l moves
+      // chunk l % CH of rows l / CH, l / CH + 32 / CH, ... The V rows of slots without a
+      // key are zero-filled (their P is 0, and 0 * NaN is not 0); their K rows are not
+      // fetched at all (their scores are masked).
+      static_assert(32 % CH == 0, "a row's 16-byte chunks must tile a warp");
+      const int c = lane % CH;
       for (int grp = 0; grp < ngroups; ++grp) {
         if ((tma_mask >> grp) & 1u) continue;
-        for (int idx = lane; idx < BR * CH; idx += 32) {
-          const int rr = idx / CH, c = idx % CH;
-          const int row = grp * BR + rr;
+        for (int row = grp * BR + lane / CH; row < (grp + 1) * BR; row += 32 / CH) {
           const int key = sink_slot_key(sl_p, bk->sinks, slot0 + row);
-          const uint32_t src_bytes = key >= 0 ? 16u : 0u;
           const size_t koff = static_cast<size_t>(key >= 0 ? key : 0) * D + c * 8;
-          cp_async16(smem_u32(dK + sw128_offset(row, c, 128)), Kbh + koff, src_bytes);
-          cp_async16(smem_u32(dV + sw128_offset(row, c, 128)), Vbh + koff, src_bytes);
+          const uint32_t so = sw128_offset(row, c, 128);
+          if (key >= 0) cp_async16(smem_u32(dK + so), Kbh + koff, 16u);
+          cp_async16(smem_u32(dV + so), Vbh + koff, key >= 0 ? 16u : 0u);
         }
       }
       if (defer) {
@@ -356,7 +359,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     auto key_of = [&](int i) { return s_key[i]; };
     int* s_wide = reinterpret_cast<int*>(sK + 4096);          // 11-bit first-pass histogram
     static_assert((RG + 1) * D * 4 <= 4096, "qbar partials overlap the top-C histogram");
-    if (a.nb <= 4 * kDecThreads) block_topk_small<4>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk, s_wide);
+    if (a.nb <= 2 * kDecThreads) cta_topk_linear(s_key, a.nb, a.C, bk->blk, a.C, s_wide, bk->tk);
+    else if (a.nb <= 4 * kDecThreads) block_topk_small<4>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk, s_wide);
     else if (a.nb <= 8 * kDecThreads) block_topk_small<8>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk, s_wide);
     else block_topk_ascending(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
     __syncthreads();

@@ -395,4 +395,206 @@ __device__ void block_topk_small(KeyFn key_of, int n, int k, int32_t* out, int c
   block_topk_small_regs<KPT>(key, n, k, out, cap, sm, nullptr, wide);
 }
 
+// Top-k of float order keys (float_order_key) over the whole CTA, two keys per thread:
+// the k largest of s_keys[0 .. n), n <= 2 * blockDim.x, with the same result as
+// block_topk_small_regs (ties at the threshold go to the lowest indices; out[0 .. k)
+// ascending, -1 in out[k .. cap)). blockDim.x must be a multiple of 32 and at least 256;
+// s_keys must be readable (8-byte aligned) up to 2 * blockDim.x entries. Every thread of
+// the CTA calls it; out is complete after the caller's next CTA barrier.
+// The first pass counts the keys in 2048 bins LINEAR in the scores' value between their
+// minimum and maximum. The bin is a monotone function of the value, so every key of a
+// higher bin is strictly larger; where the bin that holds the threshold holds exactly
+// the keys still wanted (the common case: evenly spread scores leave one or two keys in
+// that bin), the selection is settled by this one pass. Otherwise the keys of that bin
+// are ranked exactly by 8-bit radix passes over their order keys relative to the bin's
+// smallest key. Prefix counts use ballots and per-warp totals, so the whole selection
+// costs five CTA barriers when the first pass settles it.
+// fine: 2048 ints of shared memory (16-byte aligned).
+template <bool FLOAT_IN = false>
+__device__ void cta_topk_linear(const uint32_t* s_keys, int n, int k, int32_t* out, int cap, int* fine,
+                                TopkShared& sm) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nw = nt >> 5;
+  k = min(k, n);
+  if (k <= 0 || k >= n) {
+    for (int i = tid; i < cap; i += nt) out[i] = (i < k) ? i : -1;
+    return;
+  }
+  // ---- keys, minimum and maximum; the histogram is cleared meanwhile
+  const int i0 = 2 * tid;
+  const uint2 kv = reinterpret_cast<const uint2*>(s_keys)[tid];
+  uint32_t key0 = kv.x, key1 = kv.y;
+  if (FLOAT_IN) {
+    key0 = float_order_key(__uint_as_float(key0));
+    key1 = float_order_key(__uint_as_float(key1));
+  }
+  const bool p0 = i0 < n, p1 = i0 + 1 < n;
+  uint32_t kmin = min(p0 ? key0 : 0xFFFFFFFFu, p1 ? key1 : 0xFFFFFFFFu);
+  uint32_t kmax = max(p0 ? key0 : 0u, p1 ? key1 : 0u);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  if (lane == 0) {
+    sm.w_gt[warp] = static_cast<int>(kmin);
+    sm.w_eq[warp] = static_cast<int>(kmax);
+  }
+  for (int i = tid; i < 2048 / 4; i += nt) reinterpret_cast<int4*>(fine)[i] = make_int4(0, 0, 0, 0);
+  __syncthreads();
+  for (int w = 0; w < nw; ++w) {
+    kmin = min(kmin, static_cast<uint32_t>(sm.w_gt[w]));
+    kmax = max(kmax, static_cast<uint32_t>(sm.w_eq[w]));
+  }
+  // ---- linear value bins (bin 0 for every key when the span is zero or not finite)
+  const float vmin = order_key_to_float(kmin);
+  const float vspan = order_key_to_float(kmax) - vmin;
+  const float scale = (vspan > 0.f && vspan <= 3.0e38f) ? 2048.f / vspan : 0.f;
+  auto bin_of = [&](uint32_t key) {
+    return static_cast<int>(fminf((order_key_to_float(key) - vmin) * scale, 2047.f));
+  };
+  const int b0 = p0 ? bin_of(key0) : -1, b1 = p1 ? bin_of(key1) : -1;
+  if (p0) atomicAdd(&fine[b0], 1);
+  if (p1) atomicAdd(&fine[b1], 1);
+  __syncthreads();
+  // ---- the bin holding the k-th largest: thread u < 256 owns bins 2047 - 8u .. 2040 - 8u
+  {
+    int c[8];
+    if (tid < 256) {
+      const int4 hq = reinterpret_cast<const int4*>(fine)[511 - 2 * tid];
+      const int4 lq = reinterpret_cast<const int4*>(fine)[510 - 2 * tid];
+      c[0] = hq.w; c[1] = hq.z; c[2] = hq.y; c[3] = hq.x;
+      c[4] = lq.w; c[5] = lq.z; c[6] = lq.y; c[7] = lq.x;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) c[j] = 0;
+    }
+    const int own = ((c[0] + c[1]) + (c[2] + c[3])) + ((c[4] + c[5]) + (c[6] + c[7]));
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) sm.s_warp[warp] = incl;
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) incl += sm.s_warp[w];
+    const int excl = incl - own;
+    if (excl < k && incl >= k) {       // exactly one thread
+      int rem = k - excl, pb = 2047 - 8 * tid, cnt = c[0];
+#pragma unroll
+      for (int j = 0; j < 7; ++j) {
+        if (rem <= cnt) break;
+        rem -= cnt;
+        --pb;
+        cnt = c[j + 1];
+      }
+      sm.prefix = static_cast<uint32_t>(pb);
+      sm.remaining = rem;
+      sm.mask = static_cast<uint32_t>(cnt);
+    }
+    __syncthreads();
+  }
+  const int pb = static_cast<int>(sm.prefix);
+  int remaining = sm.remaining;
+  bool whole = static_cast<int>(sm.mask) == remaining;
+  // ---- exact ranking inside bin pb (hi = 32: no prefix; there the keys of bin pb all tie)
+  int hi = 32;
+  uint32_t P = 0u, cmin = 0u;
+  const bool refine = !whole;
+  if (refine) {
+    const bool c0 = b0 == pb, c1 = b1 == pb;
+    uint32_t lmin = min(c0 ? key0 : 0xFFFFFFFFu, c1 ? key1 : 0xFFFFFFFFu);
+    uint32_t lmax = max(c0 ? key0 : 0u, c1 ? key1 : 0u);
+    lmin = __reduce_min_sync(0xffffffffu, lmin);
+    lmax = __reduce_max_sync(0xffffffffu, lmax);
+    if (lane == 0) {
+      sm.w_gt[warp] = static_cast<int>(lmin);
+      sm.w_eq[warp] = static_cast<int>(lmax);
+    }
+    __syncthreads();
+    cmin = 0xFFFFFFFFu;
+    uint32_t cmax = 0u;
+    for (int w = 0; w < nw; ++w) {
+      cmin = min(cmin, static_cast<uint32_t>(sm.w_gt[w]));
+      cmax = max(cmax, static_cast<uint32_t>(sm.w_eq[w]));
+    }
+    hi = 32 - __clz(cmax - cmin);      // 0: the candidates are equal, lowest indices win
+    while (hi > 0 && !whole) {
+      const int lo = max(0, hi - 8);
+      __syncthreads();                 // the previous pass's histogram has been read
+      for (int i = tid; i < 256; i += nt) sm.hist[i] = 0;
+      __syncthreads();
+      const uint32_t r0 = key0 - cmin, r1 = key1 - cmin;
+      const uint32_t dmask = (1u << (hi - lo)) - 1u;
+      if (c0 && (hi >= 32 || (r0 >> hi) == P)) atomicAdd(&sm.hist[(r0 >> lo) & dmask], 1);
+      if (c1 && (hi >= 32 || (r1 >> hi) == P)) atomicAdd(&sm.hist[(r1 >> lo) & dmask], 1);
+      __syncthreads();
+      // every warp finds the same digit; lane l owns digits 255 - 8l .. 248 - 8l
+      int c[8], pre[8];
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) c[jj] = sm.hist[255 - 8 * lane - jj];
+      pre[0] = c[0];
+#pragma unroll
+      for (int jj = 1; jj < 8; ++jj) pre[jj] = pre[jj - 1] + c[jj];
+      int incl = pre[7];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      const int excl = incl - pre[7];
+      const int L = __ffs(__ballot_sync(0xffffffffu, incl >= remaining)) - 1;
+      int jsel = 0;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) jsel += (excl + pre[jj] < remaining) ? 1 : 0;
+      int before = excl, cnt = 0;
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        before += (jj < jsel) ? c[jj] : 0;
+        cnt = (jj == jsel) ? c[jj] : cnt;
+      }
+      const int digit = __shfl_sync(0xffffffffu, 255 - 8 * lane - jsel, L);
+      cnt = __shfl_sync(0xffffffffu, cnt, L);
+      remaining -= __shfl_sync(0xffffffffu, before, L);
+      whole = (cnt == remaining);
+      P = (P << (hi - lo)) | static_cast<uint32_t>(digit);
+      hi = lo;
+    }
+  }
+  // ---- output: selected = bin > pb, or bin == pb with prefix > P, or the first `remaining`
+  // keys (in index order) of bin pb with prefix == P; positions from ballots
+  const int take_eq = remaining;
+  auto classify = [&](uint32_t key, int b, bool& g, bool& e) {
+    const uint32_t v = (hi >= 32) ? 0u : ((key - cmin) >> hi);
+    g = b > pb || (b == pb && v > P);
+    e = b == pb && v == P;
+  };
+  bool g0, e0, g1, e1;
+  classify(key0, b0, g0, e0);
+  classify(key1, b1, g1, e1);
+  const unsigned G0 = __ballot_sync(0xffffffffu, g0), G1 = __ballot_sync(0xffffffffu, g1);
+  const unsigned E0 = __ballot_sync(0xffffffffu, e0), E1 = __ballot_sync(0xffffffffu, e1);
+  if (refine) __syncthreads();         // every thread has read the refinement's per-warp values
+  if (lane == 0) {
+    sm.w_gt[warp] = __popc(G0) + __popc(G1);
+    sm.w_eq[warp] = __popc(E0) + __popc(E1);
+  }
+  __syncthreads();
+  const unsigned lt = (1u << lane) - 1u;
+  int gtb = __popc(G0 & lt) + __popc(G1 & lt), eqb = __popc(E0 & lt) + __popc(E1 & lt);
+  for (int w = 0; w < warp; ++w) {
+    gtb += sm.w_gt[w];
+    eqb += sm.w_eq[w];
+  }
+  if (g0 || (e0 && eqb < take_eq)) {
+    const int pos = gtb + min(eqb, take_eq);
+    if (pos < cap) out[pos] = i0;
+  }
+  gtb += g0 ? 1 : 0;
+  eqb += e0 ? 1 : 0;
+  if (g1 || (e1 && eqb < take_eq)) {
+    const int pos = gtb + min(eqb, take_eq);
+    if (pos < cap) out[pos] = i0 + 1;
+  }
+  for (int i = k + tid; i < cap; i += nt) out[i] = -1;
+}
+
 }  // namespace focus

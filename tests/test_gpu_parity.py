@@ -451,6 +451,66 @@ def test_sparse_fused_matches_oracle_and_two_calls(F, case):
     assert F.device_error() == 0
 
 
+# ------------------------------------------------------------------ fused top-C on chosen relevance values
+# Every active query row is e_0, so q_bar = e_0 and R_j = kbar[j, 0] / sqrt(d) exactly up to
+# one monotone rounding: the block scores are set directly. The patterns reach the exact
+# ranking passes inside one value bin, ties at the threshold (lowest indices win), the
+# all-equal case, and scores of both signs; nb = 500 takes the one-warp selection and
+# nb = 700 the CTA-wide one.
+def _top_c_scores(pattern, nb, C, rng):
+    if pattern == "outlier_cluster":          # one far outlier: all other scores share a bin
+        v = -0.5 + np.arange(nb) * 2.0 ** -9
+        v[nb // 3] = 1.0e6
+    elif pattern == "ties_at_boundary":       # groups of seven equal scores, shuffled
+        v = np.floor(rng.permutation(nb) / 7.0) - 20.0
+    elif pattern == "all_equal":
+        v = np.full(nb, 0.5)
+    elif pattern == "near_tie_cluster":       # the C-th score inside a tight cluster
+        v = rng.uniform(-1.0, 1.0, nb)
+        idx = rng.permutation(nb)
+        v[idx[:C - 11]] = rng.uniform(50.0, 100.0, C - 11)
+        v[idx[C - 11:C + 29]] = 2.0 + np.arange(40) * 2.0 ** -16
+    else:
+        raise ValueError(pattern)
+    return v.astype(np.float32)
+
+
+@pytest.mark.parametrize("nb", [500, 700])
+@pytest.mark.parametrize("pattern", ["outlier_cluster", "ties_at_boundary", "all_equal", "near_tie_cluster"])
+def test_fused_top_c_chosen_scores(F, pattern, nb):
+    B, Hq, Hkv, G, bs, C, S, acap, d = 1, 2, 2, 32, 64, 64, 8, 32, 128
+    P = nb * bs
+    L, g0, g1 = P + G, P, P + G
+    rng = np.random.default_rng(nb + len(pattern))
+    Qh = np.zeros((B, Hq, acap, d), dtype=np.float32)
+    Qh[..., 0] = 1.0
+    Q = torch.from_numpy(Qh).to(torch.bfloat16).to(DEV)
+    n_act = [29]
+    n_active = torch.tensor(n_act, dtype=torch.int32, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=nb + 7, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=nb + 8, device=DEV)
+    kb = np.zeros((B, Hkv, nb, d), dtype=np.float32)
+    for h in range(Hkv):
+        kb[0, h, :, 0] = _top_c_scores(pattern, nb, C, rng)
+    kbar = torch.from_numpy(kb).to(DEV)
+    sinks = torch.from_numpy(np.sort(np.stack([np.stack([rng.choice(L, S, replace=False) for _ in range(Hkv)])
+                                                for _ in range(B)]), axis=-1).astype(np.int32)).to(DEV)
+    blocks_f = _i32((B, Hkv, C))
+    O_f = torch.full((B, Hq, acap, d), 4.0, dtype=torch.bfloat16, device=DEV)
+    F.focus_sparse_attention_fused(Q, n_active, K, V, kbar, C, sinks, bs, P, g0, g1, blocks_f, O_f)
+    blocks_2 = _i32((B, Hkv, C))
+    F.focus_block_select(Q, n_active, kbar, C, blocks_2)
+    torch.cuda.synchronize()
+    ref_blocks, _ = orc.block_select(inputs.to_f64(Q), n_act, kb.astype(np.float64), C)
+    assert np.array_equal(blocks_f.cpu().numpy(), ref_blocks), "fused top-C differs from the oracle"
+    assert np.array_equal(blocks_2.cpu().numpy(), ref_blocks), "focus_block_select differs from the oracle"
+    Q64, K64, V64 = inputs.to_f64(Q), inputs.to_f64(K), inputs.to_f64(V)
+    ref = orc.sparse_attention(Q64, n_act, K64, V64, sinks.cpu().numpy(), ref_blocks, bs, P, g0, g1,
+                               float(np.float32(1 / math.sqrt(d))))
+    assert_attention_close(O_f, ref, rows_valid=n_act, what=f"fused sparse ({pattern}, nb={nb})")
+    assert F.device_error() == 0
+
+
 # ------------------------------------------------------------------ the step sequencer, plain and variants
 @pytest.mark.parametrize("variant", ["plain_fused", "dream_tail_focus_meanq_ratio"])
 def test_sparse_step_sequencer(F, variant):
