@@ -238,6 +238,32 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   // stages; after that every CTA claims the next tile from the counter in CTA 0.
   // The counter's initialisation is ordered before any claim by a cluster barrier: the
   // relevance prologue's own, else a split barrier around the prologue.
+  // Pipeline barriers and the tensor-map prefetch (producer warp, lane 0).
+  auto init_pipeline = [&]() {
+    if (lane == 0) {
+      for (int st = 0; st < STAGES; ++st) {
+        mbar_init(&bk->full[st], 1);
+        mbar_init(&bk->empty[st], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bk->s_full[i], 1);
+        mbar_init(&bk->s_free[i], kDecSoftmaxWarps);
+        mbar_init(&bk->p_full[i], kDecSoftmaxWarps);
+        mbar_init(&bk->pv_done[i], 1);
+      }
+      mbar_init(&bk->drain, 1);
+      if (!FUSED) bk->abort_flag = 0;   // the relevance prologue sets it itself
+      fence_mbar_init();
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
+  };
+  if (FUSED && warp == kDecProducerWarp) {
+    // The relevance prologue does not touch these barriers: they are set up (and the sink
+    // list fetched) now, off the path from the top-C to the first tile.
+    init_pipeline();
+    if (SPARSE) pf.s0 = (snk_g && lane < a.S) ? snk_g[lane] : -1;
+  }
   if (threadIdx.x == 0 && rank == 0) bk->tile_ctr = static_cast<uint32_t>(cs * STAGES);
   if (!FUSED && cs > 1) cluster_arrive();
   if (FUSED) {
@@ -368,25 +394,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       for (int i = threadIdx.x; i < a.C; i += kDecThreads) a.blocks_out[static_cast<size_t>(bh) * a.C + i] = bk->blk[i];
   }
   if (warp == kDecProducerWarp) {
-    if (lane == 0) {
-      for (int st = 0; st < STAGES; ++st) {
-        mbar_init(&bk->full[st], 1);
-        mbar_init(&bk->empty[st], 1);
-      }
-      for (int i = 0; i < 2; ++i) {
-        mbar_init(&bk->s_full[i], 1);
-        mbar_init(&bk->s_free[i], kDecSoftmaxWarps);
-        mbar_init(&bk->p_full[i], kDecSoftmaxWarps);
-        mbar_init(&bk->pv_done[i], 1);
-      }
-      mbar_init(&bk->drain, 1);
-      if (!FUSED) bk->abort_flag = 0;   // the relevance prologue set it already
-      fence_mbar_init();
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-    }
-    if (SPARSE) {
-      if (FUSED) pf = layout_prefetch(blk_g, a.C, snk_g, a.S);
+    if (!FUSED) init_pipeline();
+    if (SPARSE && FUSED) {
+      sl_p = fused_block_layout(bk->blk, min(a.C, a.nb), a.S, a.P, a.bs, a.gen_pad, a.box_rows, a.pad_div,
+                                kDecMaxBlocks, kDecMaxSinks, &bk->sl);
+    } else if (SPARSE) {
       sl_p = build_block_layout(pf, blk_g, a.C, a.S, a.P, a.bs, a.gen_pad, a.box_rows, a.pad_div, bk->blk,
                                 kDecMaxBlocks, kDecMaxSinks, &bk->sl);
     } else {

@@ -88,6 +88,26 @@ __device__ __forceinline__ SlotLayout build_block_layout(const LayoutPrefetch& p
   return sl;
 }
 
+// The same layout when the kept-block list is already in s_blk, complete and ascending
+// with nvb valid entries first (the fused kernel's own top-C): no list walk, one load.
+__device__ __forceinline__ SlotLayout fused_block_layout(const int* s_blk, int nvb, int S, int P, int bs,
+                                                         int gen_pad, int box_rows, const FastDiv& pad_div,
+                                                         int max_blocks, int max_sinks, SlotLayout* out) {
+  const int lane = threadIdx.x & 31;
+  nvb = min(max(nvb, 0), max_blocks);
+  SlotLayout sl;
+  sl.pad_bs = (bs + 7) & ~7;
+  sl.nvb = nvb;
+  sl.last_size = nvb > 0 ? min(bs, P - s_blk[nvb - 1] * bs) : bs;
+  sl.n_sinks = min(S, max_sinks);
+  sl.gen_start = (sl.n_sinks + box_rows - 1) & ~(box_rows - 1);
+  sl.blk_start = sl.gen_start + gen_pad;
+  sl.n_slots = sl.blk_start + nvb * sl.pad_bs;
+  sl.pad_div = pad_div;
+  if (lane == 0) *out = sl;
+  return sl;
+}
+
 // Sink slots of (b, h), by one warp after build_block_layout: s_sinks[i], i < sl.n_sinks,
 // is sink i, or -1 when it is dropped -- out of range, inside the current block [g0, g1),
 // a repeat of the previous entry (the list is ascending among its valid entries) or
