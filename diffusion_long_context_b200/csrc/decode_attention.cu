@@ -112,6 +112,16 @@ __device__ __forceinline__ bool dec_wait_drain(uint64_t* bar, uint32_t parity) {
 
 constexpr int kDecMaxNb = 4096;   // fused relevance scores held in the P buffers
 
+// Top-C for more than 2 * kDecThreads blocks: out of line, so that the fused kernel's
+// straight-line prologue stays short (it runs once per launch from a cold instruction cache).
+__device__ __noinline__ void dec_top_c_large(const uint32_t* s_key, int nb, int C, int32_t* blk, TopkShared& tk,
+                                             int* s_wide) {
+  auto key_of = [&](int i) { return s_key[i]; };
+  if (nb <= 4 * kDecThreads) block_topk_small<4>(key_of, nb, C, blk, C, tk, s_wide);
+  else if (nb <= 8 * kDecThreads) block_topk_small<8>(key_of, nb, C, blk, C, tk, s_wide);
+  else block_topk_ascending(key_of, nb, C, blk, C, tk);
+}
+
 template <int NQ, int STAGES, bool SPARSE, bool FUSED>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -382,13 +392,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     if (cs > 1) cluster_sync();   // every CTA holds all nb keys
     else __syncthreads();
-    auto key_of = [&](int i) { return s_key[i]; };
     int* s_wide = reinterpret_cast<int*>(sK + 4096);          // 11-bit first-pass histogram
     static_assert((RG + 1) * D * 4 <= 4096, "qbar partials overlap the top-C histogram");
     if (a.nb <= 2 * kDecThreads) cta_topk_linear(s_key, a.nb, a.C, bk->blk, a.C, s_wide, bk->tk);
-    else if (a.nb <= 4 * kDecThreads) block_topk_small<4>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk, s_wide);
-    else if (a.nb <= 8 * kDecThreads) block_topk_small<8>(key_of, a.nb, a.C, bk->blk, a.C, bk->tk, s_wide);
-    else block_topk_ascending(key_of, a.nb, a.C, bk->blk, a.C, bk->tk);
+    else dec_top_c_large(s_key, a.nb, a.C, bk->blk, bk->tk, s_wide);
     __syncthreads();
     if (rank == 0 && a.blocks_out)
       for (int i = threadIdx.x; i < a.C; i += kDecThreads) a.blocks_out[static_cast<size_t>(bh) * a.C + i] = bk->blk[i];

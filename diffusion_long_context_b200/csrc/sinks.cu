@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kSinkThreads, 2) sink_topk_cluster_kernel(cons
   int32_t* s_cidx = reinterpret_cast<int32_t*>(s_ckey + static_cast<size_t>(gridDim.x) * S);
   int32_t* s_pos = s_cidx + static_cast<size_t>(gridDim.x) * S;  // [S] positions chosen by CTA 0
   int* s_priv = reinterpret_cast<int*>(s_pos + S);           // per-warp histograms
+  int* s_wide = s_priv + 2 * (kSinkThreads / 32) * 257;      // [2048 + 64] 11-bit first-pass histogram
   __shared__ TopkShared tk;
   const int cs = gridDim.x, rank = blockIdx.x;
   const int bh = blockIdx.y;
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kSinkThreads, 2) sink_topk_cluster_kernel(cons
 #pragma unroll
   for (int j = 0; j < KPT; ++j)
     if (i0 + j < n) s_key[i0 + j] = key[j];
-  block_topk_small_regs<KPT>(key, n, S, s_loc, S, tk, s_priv);
+  block_topk_small_regs<KPT>(key, n, S, s_loc, S, tk, s_priv, s_wide);
   __syncthreads();
   const uint32_t ck0 = smem_u32(s_ckey), ci0 = smem_u32(s_cidx);
   for (int i = threadIdx.x; i < S; i += blockDim.x) {
@@ -131,9 +132,9 @@ __global__ void __launch_bounds__(kSinkThreads, 2) sink_topk_cluster_kernel(cons
   if (rank != 0) return;
   const int nc = cs * S;
   auto ckey = [&](int i) { return s_ckey[i]; };
-  if (nc <= kSinkThreads) block_topk_small<1>(ckey, nc, S, s_pos, S, tk);
-  else if (nc <= 2 * kSinkThreads) block_topk_small<2>(ckey, nc, S, s_pos, S, tk);
-  else block_topk_small<4>(ckey, nc, S, s_pos, S, tk);
+  if (nc <= kSinkThreads) block_topk_small<1>(ckey, nc, S, s_pos, S, tk, s_wide);
+  else if (nc <= 2 * kSinkThreads) block_topk_small<2>(ckey, nc, S, s_pos, S, tk, s_wide);
+  else block_topk_small<4>(ckey, nc, S, s_pos, S, tk, s_wide);
   __syncthreads();
   int32_t* out = sinks + static_cast<size_t>(bh) * S;
   for (int i = threadIdx.x; i < S; i += blockDim.x) out[i] = s_cidx[s_pos[i]];
@@ -158,7 +159,8 @@ extern "C" int focus_sink_identify(const float* colsum, int B, int Hkv, int L, i
     if (L - (cs - 1) * chunk >= S) {
       const int vec = ((reinterpret_cast<uintptr_t>(colsum) & 15u) == 0 && (L & 3) == 0) ? 1 : 0;
       const size_t smem =
-          (static_cast<size_t>(chunk) + S + 2 * static_cast<size_t>(cs) * S + S + 2 * (kSinkThreads / 32) * 257) * 4;
+          (static_cast<size_t>(chunk) + S + 2 * static_cast<size_t>(cs) * S + S + 2 * (kSinkThreads / 32) * 257 +
+           2048 + 64) * 4;
       cudaError_t e;
       if (chunk <= 8 * kSinkThreads) {
         auto kern = sink_topk_cluster_kernel<8>;
