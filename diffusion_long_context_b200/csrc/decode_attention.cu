@@ -775,8 +775,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
   const int qpc = (n_rows + cs - 1) / cs;
   // lane: dims 4*lane .. 4*lane+3; warp: queries rank*qpc + warp + 8k, two per batch. A
-  // batch's partials are all requested before any is used; after its last batch a warp
-  // arrives on the cluster barrier (its reads are done) and waits on it only at the end.
+  // batch's partials are all requested before any is used. Every warp arrives on the
+  // cluster barrier once the values of all its remote loads have been used (so the loads
+  // are complete and nothing needs publishing: a relaxed arrive), and waits on it at the
+  // very end.
   const uint32_t po = smem_u32(part_o), pm = smem_u32(part_ml);
   auto load_q = [&](int q, bool v, float4 (&ov)[8], float2 (&ml)[8]) {
 #pragma unroll
@@ -820,7 +822,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     *reinterpret_cast<uint2*>(a.O + row * D + 4 * lane) = pk;
     if (lane == 0 && a.lse_out && i < nq_b) a.lse_out[row] = M + __log2f(l);
   };
-  bool arrived = false;
   if (warp < kDecSoftmaxWarps) {
     constexpr int W = kDecSoftmaxWarps;
     for (int qi0 = warp; qi0 < qpc; qi0 += 2 * W) {
@@ -830,16 +831,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       float2 mla[8], mlb[8];
       load_q(qa, va, ova, mla);
       load_q(qb, vb, ovb, mlb);
-      if (cs > 1 && qi0 + 2 * W >= qpc) {
-        cluster_arrive();              // this warp's reads of the partials are done
-        arrived = true;
-      }
       if (va) finish_q(qa, ova, mla);
       if (vb) finish_q(qb, ovb, mlb);
     }
   }
   if (cs > 1) {
-    if (!arrived) cluster_arrive();
+    cluster_arrive_relaxed();        // this warp's reads of the partials are done
     cluster_wait();                  // no CTA leaves while its partials may still be read
   }
 }

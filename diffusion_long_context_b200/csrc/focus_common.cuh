@@ -253,6 +253,11 @@ __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// Arrive without release semantics: for a thread whose earlier shared-memory accesses need
+// not be published, e.g. after the values of its remote loads have been consumed.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 // Atomic add on a 32-bit word of CTA `rank`'s shared memory; returns the old value.
 __device__ __forceinline__ uint32_t dsmem_atomic_add(uint32_t local_saddr, uint32_t rank, uint32_t v) {
   uint32_t old;
