@@ -396,6 +396,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     static_assert((RG + 1) * D * 4 <= 4096, "qbar partials overlap the top-C histogram");
     if (a.nb <= 2 * kDecThreads) cta_topk_linear(s_key, a.nb, a.C, bk->blk, a.C, s_wide, bk->tk);
     else dec_top_c_large(s_key, a.nb, a.C, bk->blk, bk->tk, s_wide);
+    // the K and V rings were written and read through the generic proxy above; the
+    // producer's TMA writes them next
+    fence_proxy_async_smem();
     __syncthreads();
     if (rank == 0 && a.blocks_out)
       for (int i = threadIdx.x; i < a.C; i += kDecThreads) a.blocks_out[static_cast<size_t>(bh) * a.C + i] = bk->blk[i];
@@ -714,13 +717,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (lane == 0) mbar_arrive(&bk->p_full[sb]);
     }
     n_it = it;
-    if (ok && n_it > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bk->pv_done[(n_it - 1) & 1], ((n_it - 1) >> 1) & 1, abort_flag,
-                                             a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE));
-      tc_fence_after();
-    }
-    // row sums: reduce the per-key partials over the 32 lanes of each warp (reduce-scatter),
-    // then over the four lane quadrants; the epilogue's CTA barrier orders lfin
+    // row sums (while the last PV is still running): reduce the per-key partials over the
+    // 32 lanes of each warp (reduce-scatter), then over the four lane quadrants; the
+    // epilogue's CTA barrier orders lfin
     if constexpr (QH % 32 == 0) {
       warp_sum_scatter<QH>(lsum);
 #pragma unroll
@@ -733,6 +732,11 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (threadIdx.x < NQ) {
       const int tq = threadIdx.x;
       bk->lfin[tq] = (bk->red[0][tq] + bk->red[1][tq]) + (bk->red[2][tq] + bk->red[3][tq]);
+    }
+    if (ok && n_it > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bk->pv_done[(n_it - 1) & 1], ((n_it - 1) >> 1) & 1, abort_flag,
+                                             a.dev_err, DEV_ERR_TIMEOUT_EPILOGUE));
+      tc_fence_after();
     }
     if (!ok) bk->abort_flag = 1;
   }
