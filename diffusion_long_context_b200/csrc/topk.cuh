@@ -20,6 +20,22 @@
 
 namespace focus {
 
+// Per-warp values in shared memory (one int per warp, at most 32 warps), combined by one
+// warp in parallel: lane w reads entry w and a warp reduction finishes. A serial loop over
+// the entries costs one shared-memory round trip per entry.
+__device__ __forceinline__ int warp_sum_first(const int* arr, int upto) {
+  const int lane = threadIdx.x & 31;
+  return __reduce_add_sync(0xffffffffu, lane < upto ? arr[lane] : 0);
+}
+__device__ __forceinline__ uint32_t warp_min_of(const int* arr, int n) {
+  const int lane = threadIdx.x & 31;
+  return __reduce_min_sync(0xffffffffu, lane < n ? static_cast<uint32_t>(arr[lane]) : 0xFFFFFFFFu);
+}
+__device__ __forceinline__ uint32_t warp_max_of(const int* arr, int n) {
+  const int lane = threadIdx.x & 31;
+  return __reduce_max_sync(0xffffffffu, lane < n ? static_cast<uint32_t>(arr[lane]) : 0u);
+}
+
 // Exclusive prefix sum of a 0/1 flag over the CTA in thread order; also returns the total.
 // Every thread of the CTA must call it (it synchronises the CTA).
 __device__ __forceinline__ int block_excl_scan(bool flag, int* s_warp, int& total) {
@@ -28,13 +44,8 @@ __device__ __forceinline__ int block_excl_scan(bool flag, int* s_warp, int& tota
   const int in_warp = __popc(m & ((1u << lane) - 1u));
   if (lane == 0) s_warp[warp] = __popc(m);
   __syncthreads();
-  int before = 0;
-  total = 0;
-  for (int w = 0; w < nwarps; ++w) {
-    const int c = s_warp[w];
-    if (w < warp) before += c;
-    total += c;
-  }
+  const int before = warp_sum_first(s_warp, warp);
+  total = warp_sum_first(s_warp, nwarps);
   __syncthreads();
   return before + in_warp;
 }
@@ -146,11 +157,7 @@ __device__ void block_topk_ascending(KeyFn key_of, int n, int k, int32_t* out, i
     sm.w_eq[warp] = eq;
   }
   __syncthreads();
-  int gt_before = 0, eq_before = 0;
-  for (int w = 0; w < warp; ++w) {
-    gt_before += sm.w_gt[w];
-    eq_before += sm.w_eq[w];
-  }
+  const int gt_before = warp_sum_first(sm.w_gt, warp), eq_before = warp_sum_first(sm.w_eq, warp);
   int run_eq = eq_before;
   int run_sel = gt_before + min(eq_before, take_eq);
   const unsigned lt = (1u << lane) - 1u;
@@ -222,10 +229,8 @@ __device__ void block_topk_small_regs(uint32_t (&key)[KPT], int n, int k, int32_
   if (wide)
     for (int i = tid; i < 2048 + 64; i += nt) wide[i] = 0;
   __syncthreads();
-  for (int w = 0; w < nwarps; ++w) {
-    kmin = min(kmin, static_cast<uint32_t>(sm.w_gt[w]));
-    kmax = max(kmax, static_cast<uint32_t>(sm.w_eq[w]));
-  }
+  kmin = warp_min_of(sm.w_gt, nwarps);
+  kmax = warp_max_of(sm.w_eq, nwarps);
   // relative keys rk = key - kmin in [0, range] (in place); fixed part: rk >> hi == P
   const uint32_t range = kmax - kmin;
 #pragma unroll
@@ -365,8 +370,7 @@ __device__ void block_topk_small_regs(uint32_t (&key)[KPT], int n, int k, int32_
   }
   if (lane == 31) sm.s_warp[warp] = incl;
   __syncthreads();
-  int before = incl - packed;
-  for (int w = 0; w < warp; ++w) before += sm.s_warp[w];
+  const int before = incl - packed + warp_sum_first(sm.s_warp, warp);
   int gtb = before & 0xFFFF, eqb = before >> 16;
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
@@ -439,10 +443,8 @@ __device__ void cta_topk_linear(const uint32_t* s_keys, int n, int k, int32_t* o
   }
   for (int i = tid; i < 2048 / 4; i += nt) reinterpret_cast<int4*>(fine)[i] = make_int4(0, 0, 0, 0);
   __syncthreads();
-  for (int w = 0; w < nw; ++w) {
-    kmin = min(kmin, static_cast<uint32_t>(sm.w_gt[w]));
-    kmax = max(kmax, static_cast<uint32_t>(sm.w_eq[w]));
-  }
+  kmin = warp_min_of(sm.w_gt, nw);
+  kmax = warp_max_of(sm.w_eq, nw);
   // ---- linear value bins (bin 0 for every key when the span is zero or not finite)
   const float vmin = order_key_to_float(kmin);
   const float vspan = order_key_to_float(kmax) - vmin;
@@ -475,7 +477,7 @@ __device__ void cta_topk_linear(const uint32_t* s_keys, int n, int k, int32_t* o
     }
     if (lane == 31) sm.s_warp[warp] = incl;
     __syncthreads();
-    for (int w = 0; w < warp; ++w) incl += sm.s_warp[w];
+    incl += warp_sum_first(sm.s_warp, warp);
     const int excl = incl - own;
     if (excl < k && incl >= k) {       // exactly one thread
       int rem = k - excl, pb = 2047 - 8 * tid, cnt = c[0];
@@ -510,12 +512,8 @@ __device__ void cta_topk_linear(const uint32_t* s_keys, int n, int k, int32_t* o
       sm.w_eq[warp] = static_cast<int>(lmax);
     }
     __syncthreads();
-    cmin = 0xFFFFFFFFu;
-    uint32_t cmax = 0u;
-    for (int w = 0; w < nw; ++w) {
-      cmin = min(cmin, static_cast<uint32_t>(sm.w_gt[w]));
-      cmax = max(cmax, static_cast<uint32_t>(sm.w_eq[w]));
-    }
+    cmin = warp_min_of(sm.w_gt, nw);
+    const uint32_t cmax = warp_max_of(sm.w_eq, nw);
     hi = 32 - __clz(cmax - cmin);      // 0: the candidates are equal, lowest indices win
     while (hi > 0 && !whole) {
       const int lo = max(0, hi - 8);
@@ -579,11 +577,8 @@ __device__ void cta_topk_linear(const uint32_t* s_keys, int n, int k, int32_t* o
   }
   __syncthreads();
   const unsigned lt = (1u << lane) - 1u;
-  int gtb = __popc(G0 & lt) + __popc(G1 & lt), eqb = __popc(E0 & lt) + __popc(E1 & lt);
-  for (int w = 0; w < warp; ++w) {
-    gtb += sm.w_gt[w];
-    eqb += sm.w_eq[w];
-  }
+  int gtb = __popc(G0 & lt) + __popc(G1 & lt) + warp_sum_first(sm.w_gt, warp);
+  int eqb = __popc(E0 & lt) + __popc(E1 & lt) + warp_sum_first(sm.w_eq, warp);
   if (g0 || (e0 && eqb < take_eq)) {
     const int pos = gtb + min(eqb, take_eq);
     if (pos < cap) out[pos] = i0;
