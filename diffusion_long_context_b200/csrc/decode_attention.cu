@@ -498,23 +498,23 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     bool drained_marker = !p_more;
     if (p_more) {
       const uint32_t ctr = smem_u32(&bk->tile_ctr);
-      int next = 0;
-      if (lane == 0) next = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
-      next = __shfl_sync(0xffffffffu, next, 0);
+      // Lane 0 claims the next tile right after issuing the current one; the claim (a round
+      // trip to CTA 0) is first read after the next stage wait, so it never delays a load.
+      int claim = 0;
+      if (lane == 0) claim = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
       for (int it = STAGES;; ++it) {
         const int s = it % STAGES;
         if (!__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
                                                DEV_ERR_TIMEOUT_PRODUCER)))
           break;
-        if (next >= p_n) {
+        const int tile = __shfl_sync(0xffffffffu, claim, 0);
+        if (tile >= p_n) {
           produce_end(it);
           drained_marker = true;
           break;
         }
-        const int tile = next;
-        if (lane == 0) next = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));   // claim ahead
-        next = __shfl_sync(0xffffffffu, next, 0);
         produce(it, tile, false);
+        if (lane == 0) claim = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
       }
     }
     // wait for the copies still in flight; the end marker (issue index `issued`) shares its
