@@ -358,23 +358,23 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       s_qbar[threadIdx.x] = rows > 0 ? q / static_cast<float>(rows) : 0.f;
     }
     __syncthreads();
-    // R of the staged rows: warp w scores groups of 32 rows, lane l holding dims
-    // 4l .. 4l+3 of every row of the group; a warp reduce-scatter leaves row g*32 + l's
-    // score in lane l. The order key of every score is broadcast to each CTA.
+    // R of the staged rows: warp w scores groups of 16 rows, lane l holding dims
+    // 4l .. 4l+3 of every row of the group; a warp reduce-scatter leaves row g*16 + l/2's
+    // score in lanes l and l^1. The order key of every score is broadcast to each CTA.
     const float4 qv = reinterpret_cast<const float4*>(s_qbar)[lane];
     for (int j0 = j_begin, round = 0; j0 < j_end; j0 += kKbRound, ++round) {
       const int nrow = min(kKbRound, j_end - j0);
       mbar_wait(&bk->kb_bar, round & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_PRODUCER);
-      for (int g0 = warp * 32; g0 < nrow; g0 += kDecThreads) {
-        float part[32];
+      for (int g0 = warp * 16; g0 < nrow; g0 += kDecThreads / 2) {
+        float part[16];
 #pragma unroll
-        for (int r = 0; r < 32; ++r) {
+        for (int r = 0; r < 16; ++r) {
           const float4 kv = reinterpret_cast<const float4*>(s_kb + static_cast<size_t>(g0 + r) * D)[lane];
           part[r] = (qv.x * kv.x + qv.y * kv.y) + (qv.z * kv.z + qv.w * kv.w);
         }
-        warp_sum_scatter<32>(part);
-        if (g0 + lane < nrow) {
-          const int j = j0 + g0 + lane;
+        warp_sum_scatter16(part);              // row g0 + lane / 2 in lanes 2i, 2i + 1
+        if ((lane & 1) == 0 && g0 + (lane >> 1) < nrow) {
+          const int j = j0 + g0 + (lane >> 1);
           const uint32_t key = float_order_key(part[0] * inv_sqrt_d);
           if (cs > 1) {
             for (int r = 0; r < cs; ++r)
