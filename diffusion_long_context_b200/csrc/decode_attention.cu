@@ -181,11 +181,18 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const unsigned tma_mask = __ballot_sync(0xffffffffu, key0 >= 0) & all_groups;
     if (lane == 0) mbar_expect_tx(&bk->full[s], __popc(tma_mask) * 2u * 2u * static_cast<uint32_t>(BR) * 128u);
     __syncwarp();
-    // op j: group j / 4, atom (j / 2) & 1, K for even j, V for odd j; one op per lane
+    // op j: group j / 4, atom (j / 2) & 1, K for even j, V for odd j; one op per lane. A
+    // sparse layout's group key is taken from lane grp, which looked it up above (ops
+    // j >= 32 exist only when ngroups > 8).
+    int k0a = 0, k0b = 0;
+    if (SPARSE) {
+      k0a = __shfl_sync(0xffffffffu, key0, lane >> 2);
+      k0b = __shfl_sync(0xffffffffu, key0, 8 + (lane >> 2));
+    }
     for (int j = lane; j < ngroups * 4; j += 32) {
       const int grp = j >> 2;
       if (!((tma_mask >> grp) & 1u)) continue;
-      const int k0 = group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + grp * BR);
+      const int k0 = SPARSE ? (j < 32 ? k0a : k0b) : group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + grp * BR);
       const int at = (j >> 1) & 1;
       const uint32_t off = at * (128 * 128) + grp * BR * 128;
       if (j & 1) tma_load_3d_hint(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, k0, bh, l2_stream);
