@@ -171,28 +171,37 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   // fetch tile `tile` into ring stage `it % STAGES`: TMA boxes from parallel lanes, rows
   // outside key runs by cp.async. With `defer`, a stage that used cp.async is left
   // un-arrived (returns true): the caller completes it with finish_deferred.
-  auto produce = [&](int it, int tile, bool defer) -> bool {
+  // The stage-independent part of fetching a tile (its group keys and which groups are
+  // TMA boxes), so that the producer can work it out while the tile's stage is still busy.
+  struct TilePlan {
+    unsigned tma_mask;
+    int k0a, k0b;            // group key of this lane's op j = lane and j = lane + 32
+  };
+  const unsigned all_groups = (1u << ngroups) - 1u;     // ngroups <= 16
+  auto plan_tile = [&](int tile) -> TilePlan {
+    const int slot0 = tile * 128;
+    const int key0 = (lane < ngroups) ? group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + lane * BR) : -1;
+    TilePlan pl;
+    pl.tma_mask = __ballot_sync(0xffffffffu, key0 >= 0) & all_groups;
+    // op j: group j / 4 (ops j >= 32 exist only when ngroups > 8); the key is looked up once
+    pl.k0a = __shfl_sync(0xffffffffu, key0, lane >> 2);
+    pl.k0b = __shfl_sync(0xffffffffu, key0, 8 + (lane >> 2));
+    return pl;
+  };
+  auto produce_planned = [&](int it, int tile, const TilePlan& pl, bool defer) -> bool {
     const int s = it % STAGES;
     const int slot0 = tile * 128;
     uint8_t* dK = sK + s * SM::kTile;
     uint8_t* dV = sV + s * SM::kTile;
-    const unsigned all_groups = (1u << ngroups) - 1u;     // ngroups <= 16
-    const int key0 = (lane < ngroups) ? group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + lane * BR) : -1;
-    const unsigned tma_mask = __ballot_sync(0xffffffffu, key0 >= 0) & all_groups;
+    const unsigned tma_mask = pl.tma_mask;
     if (lane == 0) mbar_expect_tx(&bk->full[s], __popc(tma_mask) * 2u * 2u * static_cast<uint32_t>(BR) * 128u);
     __syncwarp();
-    // op j: group j / 4, atom (j / 2) & 1, K for even j, V for odd j; one op per lane. A
-    // sparse layout's group key is taken from lane grp, which looked it up above (ops
-    // j >= 32 exist only when ngroups > 8).
-    int k0a = 0, k0b = 0;
-    if (SPARSE) {
-      k0a = __shfl_sync(0xffffffffu, key0, lane >> 2);
-      k0b = __shfl_sync(0xffffffffu, key0, 8 + (lane >> 2));
-    }
+    // op j: group j / 4, atom (j / 2) & 1, K for even j, V for odd j; one op per lane
+    const int k0a = pl.k0a, k0b = pl.k0b;
     for (int j = lane; j < ngroups * 4; j += 32) {
       const int grp = j >> 2;
       if (!((tma_mask >> grp) & 1u)) continue;
-      const int k0 = SPARSE ? (j < 32 ? k0a : k0b) : group_key0<SPARSE>(sl_p, bk->blk, a.bs, a.g0, slot0 + grp * BR);
+      const int k0 = j < 32 ? k0a : k0b;
       const int at = (j >> 1) & 1;
       const uint32_t off = at * (128 * 128) + grp * BR * 128;
       if (j & 1) tma_load_3d_hint(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, k0, bh, l2_stream);
@@ -233,6 +242,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     ++issued;
     return false;
   };
+  auto produce = [&](int it, int tile, bool defer) -> bool { return produce_planned(it, tile, plan_tile(tile), defer); };
   // complete the deferred stages (bit s of `stages`) once their cp.async rows have landed
   auto finish_deferred = [&](unsigned stages) {
     cp_async_wait_all();
@@ -507,20 +517,24 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const uint32_t ctr = smem_u32(&bk->tile_ctr);
       // Lane 0 claims the next tile right after issuing the current one; the claim (a round
       // trip to CTA 0) is first read after the next stage wait, so it never delays a load.
+      // The claimed tile is planned while its stage is still busy (the claim has long
+      // returned by then), so a freed stage is refilled at once.
       int claim = 0;
       if (lane == 0) claim = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
       for (int it = STAGES;; ++it) {
         const int s = it % STAGES;
+        const int tile = __shfl_sync(0xffffffffu, claim, 0);
+        TilePlan pl{0u, 0, 0};
+        if (tile < p_n) pl = plan_tile(tile);
         if (!__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
                                                DEV_ERR_TIMEOUT_PRODUCER)))
           break;
-        const int tile = __shfl_sync(0xffffffffu, claim, 0);
         if (tile >= p_n) {
           produce_end(it);
           drained_marker = true;
           break;
         }
-        produce(it, tile, false);
+        produce_planned(it, tile, pl, false);
         if (lane == 0) claim = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
       }
     }
