@@ -35,7 +35,7 @@ from diffusion_long_context_b200 import configs, inputs  # noqa: E402
 # dominant kernel on this workload, from the committed ncu summaries: the fused sparse
 # layer (default step) and the unfused sparse attention. Each is reset to None whenever
 # its kernel changes, until it is captured again.
-TRAFFIC_BYTES = {"fused": 78.61e6, "sparse": 69.53e6}
+TRAFFIC_BYTES = {"fused": 78.79e6, "sparse": 69.77e6}
 METRIC = "sparse dLLM attn step latency & active tok/s at 32K ctx; % of HBM/TC roofline"
 CFG = configs.FULL_32K
 
