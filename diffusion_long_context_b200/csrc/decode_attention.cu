@@ -17,9 +17,11 @@
 // and O^T and the row sums are rescaled. Row sums are per-thread partials reduced once
 // at the end.
 //
-// Split-KV: the CTAs of one (sequence, KV head) form a thread-block cluster, each takes a
-// contiguous share of the key tiles, and the partial results (m, l, O) are merged through
-// distributed shared memory -- no workspace and no second launch.
+// Split-KV: the CTAs of one (sequence, KV head) form a thread-block cluster. CTA r takes
+// the key tiles r, r + cs, ... for its first ring round and then claims further tiles from
+// a counter in CTA 0 (one claim in flight, planned while its stage drains); the partial
+// results (m, l, O) are merged through distributed shared memory -- no workspace and no
+// second launch. The fused form first selects the kept blocks itself (relevance + top-C).
 //
 // Warps: 0-7 softmax / epilogue (two per TMEM lane quadrant, each taking half of the
 // query columns), 8 producer (TMA for key runs, cp.async for sink rows), 9 tcgen05.mma
