@@ -9,8 +9,8 @@ Source of every definition: "Focus-dLLM: Accelerating Long-Context Diffusion LLM
 Inference via Confidence-Guided Context Focusing" (summary page of arXiv 2602.02159),
 section "方法步骤详情" (method steps), steps (1)-(5), and section "核心方法" (core
 method) for PCGI and sink-aware pruning; the English abstract on the paperdance.org
-card for cross-layer sink reuse. Readings where the pages are silent (fixed by the
-build's specification, listed in the design doc as o1..o22):
+card for cross-layer sink reuse. Readings taken where the pages are silent (numbered
+o1..o22 with the design notes):
   * PCGI candidates are the still-[MASK] positions of the current block [g0, g1).
   * k = floor(rho * n_t), clamped to the number of candidates.
   * a window of size w around p is [p - w//2, p - w//2 + w - 1], clipped to [g0, g1).
