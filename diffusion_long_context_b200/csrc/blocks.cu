@@ -2,9 +2,9 @@
 //
 // Focus-dLLM summary page, "方法步骤详情" (method steps), step (4): the prompt is cut
 // into contiguous blocks, each represented by the mean of its keys; a relevance score
-// R_b of the active queries to each block keeps the top-C blocks. Reading fixed by the
-// build's specification: R_b^h = mean over the active queries and the query heads of
-// KV group h of q . kbar_b / sqrt(d), which equals qbar_h . kbar_b / sqrt(d).
+// R_b of the active queries to each block keeps the top-C blocks. The page leaves the
+// aggregation open; the reading taken: R_b^h = mean over the active queries and the query
+// heads of KV group h of q . kbar_b / sqrt(d), which equals qbar_h . kbar_b / sqrt(d).
 #include <algorithm>
 
 #include "focus_common.cuh"
