@@ -48,6 +48,20 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(ms: float, ws: int, device) -> float:
+    """The largest of the ranks' elapsed times: the job ends with its slowest rank."""
+    if ws <= 1:
+        return ms
+    tt = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def whole_job_rate(ws: int, n_active: int, ms_per_step: float) -> float:
+    """Active tokens per second over all ranks (each rank runs its own replica)."""
+    return ws * n_active / (ms_per_step * 1e-3)
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -294,14 +308,10 @@ def run_ours(args):
             step.replay()
         t1.record()
         barrier()
-    ms_total = t0.elapsed_time(t1)
-    if ws > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(t0.elapsed_time(t1), ws, dev)
     ms_step = ms_total / args.steps
     n_act = int(step.n_active.sum().item())
-    value = ws * n_act / (ms_step * 1e-3)
+    value = whole_job_rate(ws, n_act, ms_step)
     gpu_launches = step.launches_per_step * args.steps
 
     # ---- per-call durations: each call kind of the step captured in its own CUDA graph
@@ -412,12 +422,8 @@ def run_ours(args):
         torch.cuda.current_stream().synchronize()
     x1.record()
     barrier()
-    e2e_ms = x0.elapsed_time(x1)
-    if ws > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = ws * n_act / (e2e_ms / args.steps * 1e-3)
+    e2e_ms = max_over_ranks(x0.elapsed_time(x1), ws, dev)
+    e2e_value = whole_job_rate(ws, n_act, e2e_ms / args.steps)
     h2d = conf_h.numel() * 4 + mask_h.numel()
     d2h = out_h.numel() * 2 + act_h.numel() * 4 + nact_h.numel() * 4
 

@@ -1,0 +1,75 @@
+"""The bench's multi-rank (N > 1) host logic on CPU: two gloo ranks in child processes.
+
+`bench.py --gpus N` runs one independent replica per rank (the step has no exchange
+between sequences); its only collectives are the timing barrier and the max over the
+ranks' elapsed times, and the whole-job rate counts every rank's active tokens.
+"""
+import datetime
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, ws, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(ws),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=60))
+    import bench
+    got_ws, got_rank, got_local = bench._dist()
+    elapsed = 10.0 + 5.0 * rank                       # rank r took 10 + 5 r ms
+    slowest = bench.max_over_ranks(elapsed, got_ws, torch.device("cpu"))
+    rate = bench.whole_job_rate(got_ws, 30, slowest / 10)
+    dist.barrier()
+    dist.destroy_process_group()
+    out.put((rank, got_ws, got_rank, got_local, slowest, rate))
+
+
+def test_two_ranks_report_the_slowest_rank_and_count_every_replica():
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted(out.get(timeout=120) for _ in procs)
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert [p.exitcode for p in procs] == [0, 0]
+    for rank, ws, got_rank, local, slowest, rate in res:
+        assert (ws, got_rank, local) == (2, rank, rank)
+        assert slowest == 15.0                        # both ranks see the slowest rank's time
+        assert rate == pytest.approx(2 * 30 / 1.5e-3)  # 2 replicas x 30 active tokens per 1.5 ms
+
+
+def test_single_rank_keeps_its_own_time():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.25, 1, torch.device("cpu")) == 3.25
+    assert bench.whole_job_rate(1, 30, 1.0) == pytest.approx(30_000.0)
+
+
+def test_reference_arm_prints_nothing_on_other_ranks():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1", MASTER_ADDR="127.0.0.1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
