@@ -1,10 +1,12 @@
-"""The bench's multi-rank (N > 1) host logic on CPU: two gloo ranks in child processes.
+"""The bench's host logic on CPU: the multi-rank (N > 1) path on two gloo ranks in child
+processes, and the reference arm's JSON line.
 
 `bench.py --gpus N` runs one independent replica per rank (the step has no exchange
 between sequences); its only collectives are the timing barrier and the max over the
 ranks' elapsed times, and the whole-job rate counts every rank's active tokens.
 """
 import datetime
+import json
 import os
 import socket
 import subprocess
@@ -73,3 +75,22 @@ def test_reference_arm_prints_nothing_on_other_ranks():
                        capture_output=True, text=True, env=env, timeout=300)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_reference_arm_json_line_keeps_the_contract():
+    env = dict(os.environ)
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        env.pop(k, None)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, env=env, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 1 and d["warmup"] >= 3
+    assert d["value"] > 0 and d["config"]["workload"]
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
