@@ -4,7 +4,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "focus_common.cuh"
 
@@ -18,6 +20,9 @@ constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices] = {nullptr};
 int g_sm_count[kMaxDevices] = {0};
 std::mutex g_mutex;
+// dynamic shared memory each kernel is configured for, per device ordinal
+std::mutex g_attr_mutex;
+std::map<std::pair<int, const void*>, int> g_smem_attr;
 
 int current_device() {
   int dev = 0;
@@ -60,6 +65,27 @@ int device_sm_count() {
     g_sm_count[dev] = n;
   }
   return g_sm_count[dev];
+}
+
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_attr_mutex);
+  const auto key = std::make_pair(dev, kernel);
+  const auto it = g_smem_attr.find(key);
+  if (it != g_smem_attr.end() && it->second >= bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) g_smem_attr[key] = bytes;
+  return e;
+}
+
+int configure_dynamic_smem(const void* kernel, int bytes, const char* what) {
+  const cudaError_t e = ensure_dynamic_smem(kernel, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    set_error("%s: setting %d bytes of dynamic shared memory: %s", what, bytes, cudaGetErrorString(e));
+    return FOCUS_ERR_CUDA;
+  }
+  return FOCUS_OK;
 }
 
 int* device_error_word() {

@@ -452,6 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           a.part_lse[static_cast<size_t>(split) * a.B * a.Hq * a.qcap + row_off] = lse2;
         }
       }
+    } else if (row_valid && a.n_splits > 1) {
+      // a wait ran out: this split contributes nothing, so the combine never merges a
+      // partial left in the workspace by an earlier call
+      const size_t row_off = (static_cast<size_t>(b) * a.Hq + hq) * a.qcap + qi;
+      a.part_lse[static_cast<size_t>(split) * a.B * a.Hq * a.qcap + row_off] = -INFINITY;
     }
     if (warp_active) tmem_ld_wait();
   }
@@ -800,11 +805,9 @@ int launch_attention(const AttnArgs& args, const CUtensorMap& mk, const CUtensor
                      cudaStream_t stream) {
   using SM = AttnSmem<D>;
   auto kern = attn_fwd_kernel<D, SPARSE>;
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SM::kBytes));
-    configured = true;
-  }
+  if (const int st = configure_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(SM::kBytes),
+                                            "attention kernel"))
+    return st;
   dim3 grid(args.n_splits, n_mtiles, args.B * args.Hkv);
   const cudaError_t e = launch_k(kern, grid, dim3(kThreads), SM::kBytes, stream, mk, mv, args);
   note_launch();
@@ -862,11 +865,9 @@ int launch_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat1
   c.tiles_per_cta = (total_tiles + chunks - 1) / chunks;
   chunks = (total_tiles + c.tiles_per_cta - 1) / c.tiles_per_cta;
   auto kern = colsum_kernel<D, STAGES>;
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(SM::kBytes));
-    configured = true;
-  }
+  if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(SM::kBytes),
+                                                 "colsum kernel"))
+    return st_attr;
   dim3 grid(chunks, units);
   const cudaError_t e = launch_k(kern, grid, dim3(kThreads), SM::kBytes, stream, mk, c);
   note_launch();

@@ -210,21 +210,15 @@ extern "C" int focus_block_select(const focus_bf16* Q_active, const int32_t* n_a
   while (cs < 8 && units * cs * 2 <= device_sm_count() && (nb + cs * 2 - 1) / (cs * 2) >= 16) cs *= 2;
   cudaError_t err;
   if (d == 128) {
-    static size_t cfg = 0;             // dynamic shared memory the kernel is configured for
-    if (smem > cfg) {
-      cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(std::max<size_t>(smem, 80 * 1024)));
-      cfg = std::max<size_t>(smem, 80 * 1024);
-    }
+    if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(block_select_kernel<128>),
+                            static_cast<int>(std::max<size_t>(smem, 80 * 1024)), "block_select"))
+      return st_attr;
     err = launch_k_cluster(block_select_kernel<128>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
                            n_active, kbar, Hq, Hkv, acap, acap_div, nb, C, blocks, scores_opt);
   } else {
-    static size_t cfg = 0;
-    if (smem > cfg) {
-      cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(std::max<size_t>(smem, 80 * 1024)));
-      cfg = std::max<size_t>(smem, 80 * 1024);
-    }
+    if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(block_select_kernel<64>),
+                            static_cast<int>(std::max<size_t>(smem, 80 * 1024)), "block_select"))
+      return st_attr;
     err = launch_k_cluster(block_select_kernel<64>, dim3(cs, units), dim3(kSelectThreads), smem, s, cs, q,
                            n_active, kbar, Hq, Hkv, acap, acap_div, nb, C, blocks, scores_opt);
   }

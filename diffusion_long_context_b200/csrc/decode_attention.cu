@@ -915,8 +915,11 @@ int max_active_clusters(int cs) {
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(DecSmem<NQ, STAGES>::kBytes));
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(DecSmem<NQ, STAGES>::kBytes)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, 1, 1);
   cfg.blockDim = dim3(kDecThreads);
@@ -959,8 +962,10 @@ int run_decode(const DecArgs& a0, cudaStream_t stream) {
   const int units = a.B * a.Hkv;
   const int cs = choose_cluster<NQ, STAGES, SPARSE, FUSED>(units);
   auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED>;
-  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(DecSmem<NQ, STAGES>::kBytes));
+  if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(kern),
+                                                 static_cast<int>(DecSmem<NQ, STAGES>::kBytes),
+                                                 "decode attention"))
+    return st_attr;
   const cudaError_t e =
       launch_k_cluster(kern, dim3(cs, units), dim3(kDecThreads), DecSmem<NQ, STAGES>::kBytes, stream, cs, mk, mv, a);
   note_launch();

@@ -24,6 +24,12 @@ void note_launch(int n = 1);
 int launch_status(const char* what);          // cudaGetLastError -> FOCUS_ERR_CUDA
 int device_sm_count();
 int* device_error_word();                      // device address of the error word (current device)
+// Raises the kernel's dynamic shared-memory limit to at least `bytes` on the current device.
+// The attribute is per device: the configured size is remembered per device ordinal (and
+// only once the call succeeded), so a second GPU in the process is configured on its own.
+cudaError_t ensure_dynamic_smem(const void* kernel, int bytes);
+// ensure_dynamic_smem as a status: FOCUS_OK, or FOCUS_ERR_CUDA with a message naming `what`.
+int configure_dynamic_smem(const void* kernel, int bytes, const char* what);
 
 // Error codes written to the device error word (first writer wins).
 enum DevErr : int {

@@ -164,20 +164,14 @@ extern "C" int focus_sink_identify(const float* colsum, int B, int Hkv, int L, i
       cudaError_t e;
       if (chunk <= 8 * kSinkThreads) {
         auto kern = sink_topk_cluster_kernel<8>;
-        static bool cfg8 = false;
-        if (!cfg8) {
-          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-          cfg8 = true;
-        }
+        if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(kern), 200 * 1024, "sink top-S"))
+          return st_attr;
         e = launch_k_cluster(kern, dim3(cs, B * Hkv), dim3(kSinkThreads), smem, st, cs, colsum, L, S, chunk, sinks,
                              vec);
       } else {
         auto kern = sink_topk_cluster_kernel<16>;
-        static bool cfg16 = false;
-        if (!cfg16) {
-          cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-          cfg16 = true;
-        }
+        if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(kern), 200 * 1024, "sink top-S"))
+          return st_attr;
         e = launch_k_cluster(kern, dim3(cs, B * Hkv), dim3(kSinkThreads), smem, st, cs, colsum, L, S, chunk, sinks,
                              vec);
       }
@@ -212,11 +206,9 @@ extern "C" int focus_sink_identify(const float* colsum, int B, int Hkv, int L, i
   const bool stage = stage_bytes <= kSinkStageMaxBytes && (reinterpret_cast<uintptr_t>(colsum) & 15u) == 0;
   cudaError_t e;
   if (stage) {
-    static bool cfg = false;
-    if (!cfg) {
-      cudaFuncSetAttribute(sink_topk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSinkStageMaxBytes);
-      cfg = true;
-    }
+    if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(sink_topk_kernel<true>),
+                                                   kSinkStageMaxBytes, "sink top-S"))
+      return st_attr;
     e = launch_k(sink_topk_kernel<true>, dim3(B * Hkv), dim3(1024), stage_bytes, static_cast<cudaStream_t>(stream),
                  colsum, L, S, sinks);
   } else {

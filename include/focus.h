@@ -215,10 +215,15 @@ FOCUS_API size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, int
  * (focus_sparse_workspace_bytes(...) > FOCUS_NOALLOC_SCRATCH_BYTES) returns
  * FOCUS_ERR_CAPACITY and launches nothing. The call allocates nothing.
  * The first call on a device looks the array's device address up (cudaGetSymbolAddress,
- * with that device current); make that first call before any stream capture.
+ * with that device current) and caches it per device ordinal; make that first call before
+ * any stream capture. The cached address is only valid for the device context it was
+ * taken in: after a cudaDeviceReset (or any other teardown of the primary context) it is
+ * stale, and this entry point must not be called again in that process.
  * All calls share the array and it keeps the previous call's contents; every element a
- * call reads is written earlier by the same call, so nothing has to be cleared. Calls
- * that overlap on the GPU (e.g. on two streams without ordering) race on the array.
+ * call reads is written earlier by the same call, so nothing has to be cleared (a split
+ * whose kernel gave up on a timed-out wait marks its partial empty). Calls that overlap
+ * on the GPU (e.g. on two streams without ordering) race on the array. After a call that
+ * leaves the device error word set (focus_device_error), its output is undefined.
  */
 #define FOCUS_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 

@@ -25,7 +25,9 @@ o1..o22 with the design notes):
 Everything is computed in float64 from the exact (widened) bf16 / fp32 inputs.
 Parity status: every function here is pinned by tests/test_oracle_pins.py
 (brute force, closed forms, library routines, planted structure); the composed
-step schedule is pinned only by composition of its parts.
+step schedule is pinned only by composition of its parts. The top-k margins of the
+fixed seeds (how far each selected set is from a near-tie) are recorded by
+tests/golden/make_topk_margins.py.
 """
 from __future__ import annotations
 
@@ -53,11 +55,24 @@ def top_k_ascending(scores: np.ndarray, k: int) -> np.ndarray:
 
 
 def top_k_margin(scores: np.ndarray, k: int) -> float:
-    """Gap between the k-th and (k+1)-th best score (inf if there is no (k+1)-th)."""
+    """Gap between the k-th and (k+1)-th best score: how far the kept set of a top-k is
+    from changing. inf when no score is dropped (k <= 0 or k >= n); 0 on a boundary tie,
+    where only the index order decides."""
     s = np.sort(np.asarray(scores, dtype=np.float64).reshape(-1))[::-1]
     if k <= 0 or k >= s.size:
         return math.inf
     return float(s[k - 1] - s[k])
+
+
+def top_k_relative_margin(scores: np.ndarray, k: int) -> float:
+    """top_k_margin relative to the magnitude of the k-th best score (inf as above; the
+    gap itself when the k-th score is 0)."""
+    gap = top_k_margin(scores, k)
+    if not math.isfinite(gap):
+        return gap
+    s = np.sort(np.asarray(scores, dtype=np.float64).reshape(-1))[::-1]
+    ref = abs(float(s[k - 1]))
+    return gap / ref if ref > 0.0 else gap
 
 
 # ------------------------------------------------------- step (1)+(2): PCGI + windows

@@ -52,6 +52,29 @@ def test_top_k_brute_force_with_ties():
         assert got == _brute_top_k(list(vals), k)
 
 
+def test_top_k_margin_brute_force():
+    """The margin is the gap between the worst kept and the best dropped score of the
+    brute-forced top-k (0 on a boundary tie, inf when nothing is dropped)."""
+    rng = np.random.default_rng(8)
+    for _ in range(400):
+        n = int(rng.integers(1, 9))
+        vals = rng.choice([-1.5, -0.0, 0.0, 0.25, 0.25, 1.0, 3.0, 7.5], size=n)
+        k = int(rng.integers(0, n + 1))
+        got = orc.top_k_margin(vals, k)
+        if k == 0 or k == n:
+            assert got == math.inf
+            continue
+        kept = set(_brute_top_k(list(vals), k))
+        want = min(vals[i] for i in kept) - max(vals[j] for j in range(n) if j not in kept)
+        assert got == want
+    assert orc.top_k_margin([3.0, 1.0, 2.0], 1) == 1.0
+    assert orc.top_k_margin([2.0, 2.0, 1.0], 1) == 0.0
+    assert orc.top_k_margin([0.5, -0.0, 0.0], 1) == 0.5
+    assert orc.top_k_relative_margin([4.0, 3.0, 1.0], 2) == 2.0 / 3.0
+    assert orc.top_k_relative_margin([4.0, 0.0, -1.0], 2) == 1.0
+    assert orc.top_k_relative_margin([4.0, 3.0], 2) == math.inf
+
+
 def test_top_k_golden_ties():
     g = read_golden("sink_topk_ties.txt")
     cs = np.array(_floats(g["colsum"]))
