@@ -33,11 +33,13 @@
 namespace focus {
 
 // decode_attention.cu
-bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C);
+bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C, bool sparse);
 int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                      __nv_bfloat16* O, float* lse_out, const int32_t* sinks, const int32_t* blocks, int S, int C, int bs,
                      int P, int g0, int g1, bool sparse, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
-                     cudaStream_t stream, const float* kbar = nullptr, int nb = 0, int32_t* blocks_out = nullptr);
+                     cudaStream_t stream, const float* kbar = nullptr, int nb = 0, int32_t* blocks_out = nullptr,
+                     float* colsum = nullptr, int32_t* sinks_out = nullptr, int S_out = 0,
+                     bool* sinks_done = nullptr);
 bool decode_fused_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C, int nb);
 
 constexpr int kBM = 128;            // query rows per CTA (tcgen05 M)
@@ -773,14 +775,13 @@ struct AttnPlan {
 
 // Split plan of a call. The decode kernel merges its splits inside a cluster and needs
 // workspace only for the log-sum-exp consumed by the column-sum pass.
-AttnPlan plan_attention(int B, int Hq, int Hkv, int d, int qcap, int kv_cap, bool want_lse, int L, int S, int C) {
+AttnPlan plan_attention(int B, int Hq, int Hkv, int d, int qcap, int kv_cap, bool want_lse, int L, int S, int C,
+                        bool sparse) {
   AttnPlan p{};
   const int g = Hq / Hkv;
-  if (decode_supported(d, Hq, Hkv, qcap, L, S, C)) {
-    p.decode = true;
+  if (decode_supported(d, Hq, Hkv, qcap, L, S, C, sparse)) {
+    p.decode = true;                   // merges its splits in the cluster; column sums in-kernel
     p.n_splits = 1;
-    p.lse_bytes = want_lse ? align256(static_cast<size_t>(B) * Hq * qcap * 4) : 0;
-    p.total = p.lse_bytes;
     return p;
   }
   p.n_mtiles = (g * qcap + kBM - 1) / kBM;
@@ -889,17 +890,16 @@ int run_colsum(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* 
 }
 
 template <int D, bool SPARSE>
-int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, cudaStream_t stream) {
+int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, cudaStream_t stream,
+                  int32_t* sinks_out = nullptr, int S_out = 0, bool* sinks_done = nullptr) {
   uint8_t* w = static_cast<uint8_t*>(ws);
+  if (sinks_done) *sinks_done = false;
   if (plan.decode) {
-    float* lse = plan.lse_bytes ? reinterpret_cast<float*>(w) : nullptr;
-    int st = decode_attention(args.Q, args.n_q, args.K, args.V, args.O, lse, args.sinks, args.blocks, args.S, args.C,
-                              args.bs, args.P, args.g0, args.g1, SPARSE, args.B, args.Hq, args.Hkv, args.L, args.qcap,
-                              args.scale_log2, stream);
-    if (st == FOCUS_OK && colsum)
-      st = run_colsum<D>(args.Q, args.n_q, args.K, lse, colsum, args.B, args.Hq, args.Hkv, args.L, args.qcap,
-                            args.scale_log2, stream);
-    return st;
+    // the decode kernel forms the column sums (and, where it can, the sinks) itself
+    return decode_attention(args.Q, args.n_q, args.K, args.V, args.O, nullptr, args.sinks, args.blocks, args.S,
+                            args.C, args.bs, args.P, args.g0, args.g1, SPARSE, args.B, args.Hq, args.Hkv, args.L,
+                            args.qcap, args.scale_log2, stream, nullptr, 0, nullptr, SPARSE ? nullptr : colsum,
+                            sinks_out, S_out, sinks_done);
   }
   args.box_rows = box_rows_for(SPARSE, args.L, args.bs, args.g1 - args.g0);
   args.gen_pad = gen_pad_for(args.box_rows, args.g1 - args.g0);
@@ -955,7 +955,7 @@ using namespace focus;
 
 extern "C" size_t focus_dense_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int qcap, int want_colsum) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || qcap <= 0 || Hq % Hkv) return 0;
-  return plan_attention(B, Hq, Hkv, d, qcap, L, want_colsum != 0, L, 0, 0).total;
+  return plan_attention(B, Hq, Hkv, d, qcap, L, want_colsum != 0, L, 0, 0, false).total;
 }
 
 extern "C" int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K,
@@ -972,7 +972,7 @@ extern "C" int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, co
     return FOCUS_ERR_UNSUPPORTED;
   }
   if (B == 0) return FOCUS_OK;
-  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, qcap, L, colsum_opt != nullptr, L, 0, 0);
+  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, qcap, L, colsum_opt != nullptr, L, 0, 0, false);
   FOCUS_CHECK_ARG(ws_bytes >= plan.total && (plan.total == 0 || ws), "workspace too small: need %zu bytes, got %zu",
                   plan.total, ws_bytes);
   FOCUS_CHECK_ARG((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "workspace must be 256-byte aligned");
@@ -994,6 +994,48 @@ extern "C" int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, co
                   : run_attention<64, false>(a, plan, ws, colsum_opt, s);
 }
 
+extern "C" int focus_dense_attention_sinks(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K,
+                                           const focus_bf16* V, int B, int Hq, int Hkv, int L, int d, int qcap,
+                                           float scale, focus_bf16* O, float* colsum, int S, int32_t* sinks, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  int st = check_common(Q, K, V, O, B, Hq, Hkv, L, d, qcap);
+  if (st != FOCUS_OK) return st;
+  FOCUS_CHECK_ARG(colsum && sinks, "null pointer argument");
+  FOCUS_CHECK_ARG(S >= 1 && S <= 4096, "bad S=%d", S);
+  if (d != 64 && d != 128) {
+    set_error("head dim %d unsupported (64 or 128)", d);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
+  if ((Hq / Hkv) * qcap > 256) {
+    set_error("column sums need (Hq/Hkv)*qcap <= 256, got %d", (Hq / Hkv) * qcap);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
+  if (B == 0) return FOCUS_OK;
+  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, qcap, L, true, L, 0, 0, false);
+  FOCUS_CHECK_ARG(ws_bytes >= plan.total && (plan.total == 0 || ws), "workspace too small: need %zu bytes, got %zu",
+                  plan.total, ws_bytes);
+  FOCUS_CHECK_ARG((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "workspace must be 256-byte aligned");
+  AttnArgs a{};
+  a.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  a.n_q = n_q;
+  a.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  a.V = reinterpret_cast<const __nv_bfloat16*>(V);
+  a.O = reinterpret_cast<__nv_bfloat16*>(O);
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.qcap = qcap;
+  a.g = Hq / Hkv;
+  a.scale_log2 = scale * kLog2e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bool done = false;
+  st = d == 128 ? run_attention<128, false>(a, plan, ws, colsum, s, sinks, S, &done)
+                : run_attention<64, false>(a, plan, ws, colsum, s, sinks, S, &done);
+  if (st != FOCUS_OK || done) return st;
+  return focus_sink_identify(colsum, B, Hkv, L, S, sinks, stream);   // the top-S as its own launch
+}
+
 extern "C" size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int acap, int S, int C, int bs,
                                                int P, int g0, int g1) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || acap <= 0 || Hq % Hkv || bs <= 0 || C <= 0 || S < 0) return 0;
@@ -1001,7 +1043,7 @@ extern "C" size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, in
   const int br = box_rows_for(true, L, bs, g1 - g0);
   const long kv_cap = static_cast<long>(std::min(C, std::max(nb, 0))) * ((bs + 7) & ~7) + gen_pad_for(br, g1 - g0) +
                       gen_pad_for(br, std::min(S, kMaxSinks));
-  return plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(std::min<long>(kv_cap, 1 << 30)), false, L, S, C)
+  return plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(std::min<long>(kv_cap, 1 << 30)), false, L, S, C, true)
       .total;
 }
 
@@ -1033,7 +1075,7 @@ extern "C" int focus_sparse_attention(const focus_bf16* Q_active, const int32_t*
   const long kv_cap = static_cast<long>(std::min(C, nb)) * ((bs + 7) & ~7) + gen_pad_for(br, g1 - g0) +
                       gen_pad_for(br, S);
   FOCUS_CHECK_ARG(kv_cap < (1L << 30), "key set too large");
-  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(kv_cap), false, L, S, C);
+  const AttnPlan plan = plan_attention(B, Hq, Hkv, d, acap, static_cast<int>(kv_cap), false, L, S, C, true);
   FOCUS_CHECK_ARG(ws_bytes >= plan.total && (plan.total == 0 || ws), "workspace too small: need %zu bytes, got %zu",
                   plan.total, ws_bytes);
   FOCUS_CHECK_ARG((reinterpret_cast<uintptr_t>(ws) & 255u) == 0, "workspace must be 256-byte aligned");

@@ -6,7 +6,8 @@
 //   * sparse (method steps (5)): the active queries over I_p = sinks U kept prompt
 //     blocks U current block (slot layout in slots.cuh).
 // With so few queries the 128 keys of a tile are the MMA's M dimension and the queries
-// its N dimension:
+// its N dimension (up to 64 rows of a KV group per CTA; larger groups are cut into row
+// slices, one cluster each):
 //   S^T[key, q] = K_tile . Q^T        (M = 128 keys, N = NQ queries, K = d)   -> TMEM
 //   O^T[dim, q] += V_tile^T . P^T      (M = d = 128, N = NQ, K = 128 keys)    -> TMEM
 // V_tile^T is the V tile read as an MN-major A operand; P (bf16) is written to shared
@@ -46,6 +47,11 @@ constexpr int kDecThreads = kDecSoftmaxThreads + 64;
 constexpr int kDecD = 128;
 constexpr int kDecMaxBlocks = 512;
 constexpr int kDecMaxSinks = 512;
+// Query rows per KV group the decode kernel serves: above 64 the group's rows are cut into
+// slices of 64, one cluster per slice (GQA 7:1 at 32 active queries = 4 slices). Each slice
+// streams the group's keys again (from L2 when the slices run together), so beyond a few
+// slices the 128-row tile kernel, which reads the keys once per 128 rows, is the better fit.
+constexpr int kDecMaxRows = 256;
 constexpr int kDecProducerWarp = kDecSoftmaxWarps;
 constexpr int kDecMmaWarp = kDecSoftmaxWarps + 1;
 
@@ -62,12 +68,20 @@ struct DecArgs {
   int32_t* blocks_out;         // [B, Hkv, C] kept blocks written by the fused kernel, or null
   int nb;
   int B, Hq, Hkv, L, qcap, g;
+  int n_slices;                // clusters per (b, kv head): the group's rows in slices of NQ
   int box_rows;                // rows per TMA box (divides 128)
   int gen_pad;                 // slots of the current block (multiple of box_rows)
   int S, C, bs, P, g0, g1;
   float scale_log2;
   FastDiv pad_div, bs_div, qcap_div;   // by round_up(bs, 8), bs and qcap (host-computed)
   int* dev_err;
+  // dense sink layer (column-sum form): colsum [B, Hkv, L] of the softmax rows, and
+  // optionally the top-S columns sinks_out [B, Hkv, S_out] selected by the cluster
+  float* colsum;
+  int32_t* sinks_out;
+  int S_out;
+  int ts_chunk;                // columns per CTA for the top-S (a multiple of 4)
+  int ts_kpt;                  // columns per thread for it: 8, 16 or 32
 };
 
 struct __align__(8) DecBook {
@@ -85,9 +99,17 @@ struct __align__(8) DecBook {
   int sinks[kDecMaxSinks];
   TopkShared tk;
   uint64_t kb_bar;         // kbar rows staged by bulk copy (fused relevance prologue)
+  uint64_t q_bar;          // the group's query rows staged by bulk copy (fused relevance prologue)
   uint32_t qvalid[2];      // bit q: query column q is a real query
   uint32_t tile_ctr;       // next dynamically claimed tile (CTA 0 of the cluster)
   int stage_tile[4];       // tile held by each ring stage, -1 = no more tiles
+  // column-sum pass of the sink layer: a K-only ring over the idle K ring and the part of
+  // the V ring the merge does not read
+  uint64_t c_full[6], c_empty[6], c_sfull[2], c_sfree[2];
+  int c_tile[6];           // tile held by each column-sum slot
+  int c_stile[2];          // tile whose scores an S buffer holds, -1 = end
+  uint32_t c_ctr;          // tiles claimed so far for the column-sum pass (CTA 0)
+  float lse2[64];          // log2-domain log-sum-exp of every query column (+inf: not a query)
 };
 
 template <int NQ, int STAGES>
@@ -124,12 +146,185 @@ __device__ __noinline__ void dec_top_c_large(const uint32_t* s_key, int nb, int 
   else block_topk_ascending(key_of, nb, C, blk, C, tk);
 }
 
-template <int NQ, int STAGES, bool SPARSE, bool FUSED>
+// ------------------------------------------------------------------ sink layer
+// Column sums of the dense sink layer (method steps (3): the attention distribution of the
+// sink layer, aggregated over the active queries, identifies the sinks). They run after
+// the cluster merge, once the log-sum-exp of every query is known:
+//   colsum[b, h, key] = sum over query columns q of 2^(scale_log2 * s[key, q] - lse2[q]).
+// The CTAs claim 128-key tiles from a counter in CTA 0, from the last tile down, so the
+// tiles the attention pass read last (the ones most likely still in L2: the pass loaded K
+// without the evict-first hint it gives V) come first. K tiles flow through a CS-slot ring
+// made of the K ring and the V-ring stages the merge does not read; S^T = K_tile . Q^T
+// lands in the two S buffers of tensor memory; each softmax thread owns one key, the two
+// query halves of a key are added through shared memory, and the key's sum is stored.
+template <int NQ, int STAGES>
+__device__ __noinline__ void decode_colsum_phase(const CUtensorMap* tmK, const DecArgs& a, DecBook* bk, uint8_t* sK,
+                                                 uint8_t* sV, const uint8_t* sQ, uint32_t tmem, int bh) {
+  using SM = DecSmem<NQ, STAGES>;
+  constexpr int D = kDecD;
+  constexpr int QH = NQ / 2;
+  constexpr uint32_t kPart = NQ * D * 4 + NQ * 8;              // the merge's partials, V ring start
+  constexpr int V0 = static_cast<int>((kPart + SM::kTile - 1) / SM::kTile);
+  constexpr int CS = STAGES + (STAGES > V0 ? STAGES - V0 : 0);
+  static_assert(CS >= 2 && CS <= 6, "column-sum ring");
+  const int warp = warp_id(), lane = lane_id();
+  volatile int* abort_flag = &bk->abort_flag;
+  __syncthreads();                             // lse2 of every query is in place
+  if (*abort_flag) return;                     // uniform: read after a CTA barrier
+  const int p_n = (a.L + 127) / 128;
+  const int BR = a.box_rows;                   // dense layout: boxes of BR consecutive keys
+  const int ngroups = 128 / BR;
+  auto slot_addr = [&](int sl) -> uint8_t* {
+    return sl < STAGES ? sK + sl * SM::kTile : sV + (V0 + sl - STAGES) * SM::kTile;
+  };
+  if (warp == kDecProducerWarp) {
+    if (lane == 0) {
+      const uint32_t ctr = smem_u32(&bk->c_ctr);
+      const uint64_t l2_once = l2_evict_first_policy();   // the last read of these K rows
+      for (int it = 0;; ++it) {
+        const int sl = it % CS;
+        if (it >= CS && !mbar_wait(&bk->c_empty[sl], ((it / CS) - 1) & 1, abort_flag, a.dev_err,
+                                   DEV_ERR_TIMEOUT_PRODUCER))
+          break;
+        const int tile = p_n - 1 - static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
+        if (tile < 0) {
+          bk->c_tile[sl] = -1;
+          mbar_arrive(&bk->c_full[sl]);
+          break;
+        }
+        int nbox = 0;
+        for (int grp = 0; grp < ngroups; ++grp) nbox += (tile * 128 + grp * BR < a.L) ? 1 : 0;
+        bk->c_tile[sl] = tile;
+        mbar_arrive_expect_tx(&bk->c_full[sl], static_cast<uint32_t>(nbox * 2 * BR * 128));
+        uint8_t* dK = slot_addr(sl);
+        for (int grp = 0; grp < nbox; ++grp)
+          for (int at = 0; at < 2; ++at)
+            tma_load_3d_hint(smem_u32(dK + at * (128 * 128) + grp * BR * 128), tmK, &bk->c_full[sl], at * 64,
+                             tile * 128 + grp * BR, bh, l2_once);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kDecMmaWarp) {
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(128, NQ, false, false);
+      const uint64_t q_desc = sw128_desc(smem_u32(sQ), 16, 1024);
+      for (int it = 0;; ++it) {
+        const int sl = it % CS, sb = it & 1;
+        int tile = -1;
+        if (mbar_wait(&bk->c_full[sl], (it / CS) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) tile = bk->c_tile[sl];
+        // S buffer sb (and its tile id) are free once the softmax warps are done with tile it - 2
+        if (it >= 2 && !mbar_wait(&bk->c_sfree[sb], ((it - 2) >> 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
+          tile = -1;
+        bk->c_stile[sb] = tile;
+        if (tile >= 0) {
+          tc_fence_after();
+          const uint64_t kd = sw128_desc(smem_u32(slot_addr(sl)), 16, 1024);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks)
+            mma_bf16(tmem + sb * NQ, kd + (ks >> 2) * (128 * 128 / 16) + (ks & 3) * 2,
+                     q_desc + (ks >> 2) * (NQ * 128 / 16) + (ks & 3) * 2, idesc_qk, ks > 0 ? 1u : 0u);
+          mma_commit(&bk->c_sfull[sb]);
+          mma_commit(&bk->c_empty[sl]);
+        } else {
+          mbar_arrive(&bk->c_sfull[sb]);       // stands in for the commit
+        }
+        mbar_arrive(&bk->c_sfull[sb]);         // publishes c_stile[sb]
+        if (tile < 0) break;
+      }
+    }
+    __syncwarp();
+  } else {
+    const int t = threadIdx.x & 127, q0 = (warp >> 2) * QH;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    float* hbuf = &bk->red[0][0];              // [2][128]: the second query half's sums
+    float lse[QH];
+#pragma unroll
+    for (int q = 0; q < QH; ++q) lse[q] = bk->lse2[q0 + q];
+    for (int it = 0;; ++it) {
+      const int sb = it & 1;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&bk->c_sfull[sb], (it >> 1) & 1, abort_flag, a.dev_err,
+                                                        DEV_ERR_TIMEOUT_SOFTMAX));
+      const int tile = ok ? bk->c_stile[sb] : -1;
+      if (bar_red_or(1, kDecSoftmaxThreads, tile < 0 || *abort_flag != 0)) break;
+      tc_fence_after();
+      uint32_t rg[QH];
+      tmem_ld_cols<QH>(tmem + lane_addr + sb * NQ + q0, rg);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bk->c_sfree[sb]);
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < QH; ++q) acc += exp2_approx(__uint_as_float(rg[q]) * a.scale_log2 - lse[q]);
+      if (warp >= 4) hbuf[sb * 128 + t] = acc;
+      named_bar_sync(1, kDecSoftmaxThreads);
+      const int key = tile * 128 + t;
+      if (warp < 4 && key < a.L) a.colsum[static_cast<size_t>(bh) * a.L + key] = acc + hbuf[sb * 128 + t];
+    }
+  }
+}
+
+// Top-S sinks of the sink layer's column sums, selected by the cluster (core method: the
+// sinks found at the sink layer are reused by every deeper layer). CTA r takes the
+// contiguous columns [r * chunk, r * chunk + chunk) of its (b, h), selects their top-S and
+// pushes the S candidates (order key, column) into CTA 0 in rank order, so the candidate
+// list is in ascending column order and a tie between candidates still resolves to the
+// lower column; CTA 0 selects the top-S of the cs * S candidates. `ws` is the idle K and V
+// rings. The column sums were written by the cluster's CTAs before a fence and a cluster
+// barrier; they are read from L2.
+template <int KPT>
+__device__ __forceinline__ void decode_topk_share(const float* row, int n, int S, uint32_t* s_key, int32_t* s_loc,
+                                                  TopkShared& tk, int* s_priv, int* s_wide) {
+  const int i0 = threadIdx.x * KPT;
+  uint32_t key[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) key[j] = (i0 + j < n) ? float_order_key(__ldcg(row + i0 + j)) : 0u;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    if (i0 + j < n) s_key[i0 + j] = key[j];
+  block_topk_small_regs<KPT>(key, n, S, s_loc, S, tk, s_priv, s_wide);
+}
+
+__device__ __noinline__ void decode_sink_topk(const DecArgs& a, DecBook* bk, uint8_t* ws, int bh, int rank, int cs) {
+  const int chunk = a.ts_chunk, S = a.S_out;
+  const int c0 = rank * chunk;
+  const int n = min(chunk, a.L - c0);          // >= S (host-checked)
+  uint32_t* s_key = reinterpret_cast<uint32_t*>(ws);                          // [chunk]
+  int32_t* s_loc = reinterpret_cast<int32_t*>(s_key + chunk);                 // [S]
+  uint32_t* s_ckey = reinterpret_cast<uint32_t*>(s_loc + S);                  // [cs * S] (CTA 0)
+  int32_t* s_cidx = reinterpret_cast<int32_t*>(s_ckey + static_cast<size_t>(cs) * S);
+  int32_t* s_pos = s_cidx + static_cast<size_t>(cs) * S;                      // [S]
+  int* s_priv = reinterpret_cast<int*>(s_pos + S);                            // per-warp histograms
+  int* s_wide = s_priv + 2 * (kDecThreads / 32) * 257;                        // [2048 + 64]
+  const float* row = a.colsum + static_cast<size_t>(bh) * a.L + c0;
+  if (a.ts_kpt <= 8) decode_topk_share<8>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);
+  else if (a.ts_kpt <= 16) decode_topk_share<16>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);
+  else decode_topk_share<32>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);
+  __syncthreads();
+  const uint32_t ck0 = smem_u32(s_ckey), ci0 = smem_u32(s_cidx);
+  for (int i = threadIdx.x; i < S; i += kDecThreads) {
+    const int c = s_loc[i];
+    const uint32_t slot = static_cast<uint32_t>(rank * S + i) * 4u;
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dsmem_addr(ck0 + slot, 0)), "r"(s_key[c]) : "memory");
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dsmem_addr(ci0 + slot, 0)), "r"(c0 + c) : "memory");
+  }
+  if (cs > 1) cluster_sync();                  // every candidate is in CTA 0
+  else __syncthreads();
+  if (rank != 0) return;
+  const int nc = cs * S;
+  auto ckey = [&](int i) { return s_ckey[i]; };
+  if (nc <= kDecThreads) block_topk_small<1>(ckey, nc, S, s_pos, S, bk->tk, s_wide);
+  else if (nc <= 2 * kDecThreads) block_topk_small<2>(ckey, nc, S, s_pos, S, bk->tk, s_wide);
+  else block_topk_small<4>(ckey, nc, S, s_pos, S, bk->tk, s_wide);
+  __syncthreads();
+  int32_t* out = a.sinks_out + static_cast<size_t>(bh) * S;
+  for (int i = threadIdx.x; i < S; i += kDecThreads) out[i] = s_cidx[s_pos[i]];
+}
+
+template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                       const DecArgs a) {
-  griddep_wait();               // inputs may come from the previous kernel on the stream
-  griddep_launch_dependents();
+                       const __grid_constant__ DecArgs a) {
   using SM = DecSmem<NQ, STAGES>;
   constexpr int D = kDecD;
   constexpr int CH = D / 8;
@@ -144,17 +339,22 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int warp = warp_id(), lane = lane_id();
   const int cs = gridDim.x;                    // CTAs per (b, h) == cluster size
   const int rank = blockIdx.x;
-  const int bh = blockIdx.y;
+  // cluster (blockIdx.y) = (sequence b, KV head kvh, row slice): the slice holds the
+  // group rows row0 .. row0 + n_rows - 1 (row r <-> query head kvh*g + r / qcap, position
+  // r % qcap); every slice of a group streams the same keys
+  const int bh = static_cast<int>(blockIdx.y) / a.n_slices;
+  const int row0 = (static_cast<int>(blockIdx.y) - bh * a.n_slices) * NQ;
   const int b = bh / a.Hkv, kvh = bh % a.Hkv;
-  const int nq_b = a.n_q ? min(a.n_q[b], a.qcap) : a.qcap;
-  const int n_rows = a.g * a.qcap;             // <= NQ
+  const int n_rows = min(NQ, a.g * a.qcap - row0);   // rows of this slice
   const int G = a.g1 - a.g0;
   const FastDiv qdiv = a.qcap_div;             // query column q <-> (head q / qcap, row q % qcap)
 
-  // ---------------------------------------------------------------- prologue
-  // The producer warp initialises the barriers, builds the slot layout and issues the first
-  // STAGES tiles before the CTA barrier; meanwhile the MMA warp allocates tensor memory and
-  // the other warps stage Q.
+  // ---------------------------------------------------------------- setup
+  // Work that reads no input of the call runs before the wait for the previous kernel on
+  // the stream (with programmatic dependent launch it overlaps that kernel's tail): the
+  // pipeline barriers, the tensor-map prefetch, the tile counter, the tensor-memory
+  // allocation and, in the fused form, an L2 prefetch of this CTA's share of the block
+  // means (a cache hint only: the copy that uses them is issued after the wait).
   volatile int* abort_flag = &bk->abort_flag;
   const int BR = a.box_rows;
   const int ngroups = 128 / BR;
@@ -166,7 +366,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int32_t* blk_g = FUSED ? bk->blk : a.blocks + static_cast<size_t>(bh) * a.C;
   const int32_t* snk_g = a.sinks ? a.sinks + static_cast<size_t>(bh) * a.S : nullptr;
   LayoutPrefetch pf{};
-  if (SPARSE && !FUSED && warp == kDecProducerWarp) pf = layout_prefetch(blk_g, a.C, snk_g, a.S);
   SlotLayout sl_p{};
   int p_n = 0;                 // tiles of this (b, h)
   bool p_more = true;          // the end marker is not issued yet
@@ -207,6 +406,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int at = (j >> 1) & 1;
       const uint32_t off = at * (128 * 128) + grp * BR * 128;
       if (j & 1) tma_load_3d_hint(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, k0, bh, l2_stream);
+      else if (COLSUM) tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh);   // read again below
       else tma_load_3d_hint(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh, l2_stream);
     }
     if (SPARSE && tma_mask != all_groups) {
@@ -281,37 +481,76 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mbar_init(&bk->pv_done[i], 1);
       }
       mbar_init(&bk->drain, 1);
-      if (!FUSED) bk->abort_flag = 0;   // the relevance prologue sets it itself
+      if (FUSED) {
+        mbar_init(&bk->kb_bar, 1);
+        mbar_init(&bk->q_bar, 1);
+      }
+      if (COLSUM) {
+        for (int st = 0; st < 6; ++st) {
+          mbar_init(&bk->c_full[st], 1);
+          mbar_init(&bk->c_empty[st], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+          mbar_init(&bk->c_sfull[i], 2);      // the MMAs' commit + the tile id published
+          mbar_init(&bk->c_sfree[i], kDecSoftmaxWarps);
+        }
+        if (rank == 0) bk->c_ctr = 0u;
+      }
+      bk->abort_flag = 0;
+      if (rank == 0) bk->tile_ctr = static_cast<uint32_t>(cs * STAGES);
       fence_mbar_init();
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
   };
-  if (FUSED && warp == kDecProducerWarp) {
-    // The relevance prologue does not touch these barriers: they are set up (and the sink
-    // list fetched) now, off the path from the top-C to the first tile.
+  // fused form: this CTA's contiguous share [j_begin, j_end) of the block means
+  const int kb_chunk = FUSED ? (a.nb + cs - 1) / cs : 0;
+  const int j_begin = FUSED ? min(a.nb, rank * kb_chunk) : 0;
+  const int j_end = FUSED ? min(a.nb, j_begin + kb_chunk) : 0;
+  const float* kb = FUSED ? a.kbar + static_cast<size_t>(bh) * a.nb * D : nullptr;
+  if (warp == kDecProducerWarp) {
     init_pipeline();
-    if (SPARSE) pf.s0 = (snk_g && lane < a.S) ? snk_g[lane] : -1;
+    if (FUSED && lane == 0 && j_begin < j_end)
+      bulk_prefetch_l2(kb + static_cast<size_t>(j_begin) * D, static_cast<uint32_t>((j_end - j_begin) * D * 4));
+  } else if (warp == kDecMmaWarp) {
+    tmem_alloc(&bk->tmem_base, SM::kTmemCols);
+    tmem_relinquish();
   }
-  if (threadIdx.x == 0 && rank == 0) bk->tile_ctr = static_cast<uint32_t>(cs * STAGES);
+  tc_fence_before();
+  __syncthreads();              // barriers initialised, tensor memory allocated
+  tc_fence_after();
+
+  griddep_wait();               // inputs may come from the previous kernel on the stream
+  griddep_launch_dependents();
+
+  // ---------------------------------------------------------------- prologue
+  // The producer warp builds the slot layout and issues the first STAGES tiles before the
+  // CTA barrier; meanwhile the other warps stage Q.
+  const int nq_b = a.n_q ? min(a.n_q[b], a.qcap) : a.qcap;
+  if (SPARSE && warp == kDecProducerWarp) {
+    // kept-block list and sinks of this (b, h): their first entries are fetched right away
+    if (FUSED) pf.s0 = (snk_g && lane < a.S) ? snk_g[lane] : -1;
+    else pf = layout_prefetch(blk_g, a.C, snk_g, a.S);
+  }
   if (!FUSED && cs > 1) cluster_arrive();
   if (FUSED) {
     // ---- block relevance R_b = qbar . kbar_b / sqrt(d) and top-C (method steps (4)) ----
     // This CTA scores the contiguous kbar rows [j_begin, j_end). They are staged into the
-    // (still idle) V ring by bulk copies of up to kKbRound rows, the first issued before
-    // qbar is formed; qbar's partial sums use the (still idle) K ring.
-    constexpr int kKbRound = 128;
-    static_assert(kKbRound * D * 4 <= STAGES * SM::kTile, "kbar round exceeds the V ring");
+    // (still idle) V ring by bulk copies of up to kKbRound rows; the group's query rows
+    // (contiguous in Q) are staged into the (still idle) K ring by one bulk copy issued
+    // with the first round, and qbar is summed from there.
     constexpr int RG = kDecThreads / 64;                       // qbar row groups
-    float* s_part = reinterpret_cast<float*>(sK);            // [RG][D]
-    float* s_qbar = s_part + RG * D;                           // [D]
+    constexpr int kKbRound = STAGES >= 3 ? 128 : 120;          // leaves room for the qbar partials
+    static_assert(kKbRound * D * 4 + (RG + 1) * D * 4 <= STAGES * SM::kTile, "kbar round exceeds the V ring");
+    static_assert(kDecMaxRows * D * 2 <= STAGES * SM::kTile, "the group's query rows exceed the K ring");
+    const __nv_bfloat162* s_qrows = reinterpret_cast<const __nv_bfloat162*>(sK);   // [g * qcap][D / 2]
     float* s_kb = reinterpret_cast<float*>(sV);                // [kKbRound][D]
+    float* s_part = s_kb + kKbRound * D;                       // [RG][D]
+    float* s_qbar = s_part + RG * D;                           // [D]
     uint32_t* s_key = reinterpret_cast<uint32_t*>(sP);        // [nb] order keys of R, in every CTA
     const int rows = a.g * nq_b;
     const float inv_sqrt_d = rsqrtf(static_cast<float>(D));
-    const float* kb = a.kbar + static_cast<size_t>(bh) * a.nb * D;
-    const int chunk = (a.nb + cs - 1) / cs;
-    const int j_begin = min(a.nb, rank * chunk), j_end = min(a.nb, j_begin + chunk);
+    const int nr = a.g * a.qcap;
     const uint32_t sK0 = smem_u32(s_key);
     auto issue_round = [&](int j0) {
       const int nrow = min(kKbRound, j_end - j0);
@@ -319,55 +558,44 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       bulk_load(smem_u32(s_kb), kb + static_cast<size_t>(j0) * D, static_cast<uint32_t>(nrow * D * 4), &bk->kb_bar);
     };
     if (threadIdx.x == 0) {
-      bk->abort_flag = 0;
-      mbar_init(&bk->kb_bar, 1);
-      fence_mbar_init();
+      const uint32_t qbytes = static_cast<uint32_t>(nr * D * 2);
+      mbar_arrive_expect_tx(&bk->q_bar, qbytes);
+      bulk_load(smem_u32(sK), a.Q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * a.g) * a.qcap * D,
+                qbytes, &bk->q_bar);
       if (j_begin < j_end) issue_round(j_begin);
     }
-    // qbar over the group's active rows: RG row groups x 64 dim pairs, 8 rows in flight per
-    // thread. Row slot r = (head r / qcap, position r % qcap); every slot is loaded and the
-    // positions >= nq_b are masked afterwards, so the loads do not wait for n_q.
-    const int t = threadIdx.x, dp = t % 64, rg = t / 64;
-    const int nr = a.g * a.qcap;
-    auto load8 = [&](int r0, __nv_bfloat162 (&v)[8]) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int r = r0 + RG * u;
-        v[u] = __floats2bfloat162_rn(0.f, 0.f);
-        if (r < nr) {
-          const int rh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
-          const int i = r - rh * a.qcap;
-          v[u] = *reinterpret_cast<const __nv_bfloat162*>(
-              a.Q + ((static_cast<size_t>(b) * a.Hq + kvh * a.g + rh) * a.qcap + i) * D + 2 * dp);
-        }
-      }
-    };
-    auto mask8 = [&](int r0, __nv_bfloat162 (&v)[8]) {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int r = r0 + RG * u;
-        const int rh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
-        if (r - rh * a.qcap >= nq_b) v[u] = __floats2bfloat162_rn(0.f, 0.f);
-      }
-    };
+    // qbar over the group's valid rows: RG row groups x 64 dim pairs. Row r is query head
+    // r / qcap at position i = r % qcap, valid when i < nq_b.
     {
-      __nv_bfloat162 qv8[8];
-      load8(rg, qv8);
+      const int t = threadIdx.x, dp = t % 64, rg = t / 64;
       float2 acc = make_float2(0.f, 0.f);
-      for (int r0 = rg;;) {
-        mask8(r0, qv8);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float2 f = __bfloat1622float2(qv8[u]);
+      mbar_wait(&bk->q_bar, 0, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_PRODUCER);
+      int i = rg;                                   // rg < RG <= qcap is not assumed
+      while (i >= a.qcap) i -= a.qcap;
+#pragma unroll 4
+      for (int r = rg; r < nr; r += RG) {
+        if (i < nq_b) {
+          const float2 f = __bfloat1622float2(s_qrows[r * (D / 2) + dp]);
           acc.x += f.x;
           acc.y += f.y;
         }
-        r0 += RG * 8;
-        if (r0 >= nr) break;
-        load8(r0, qv8);
+        i += RG;
+        while (i >= a.qcap) i -= a.qcap;
       }
       s_part[rg * D + 2 * dp] = acc.x;
       s_part[rg * D + 2 * dp + 1] = acc.y;
+    }
+    // this slice's rows as the MMA's K-major SW128 Q operand, from the staged copy (the
+    // fence after the top-C orders these writes before the tensor cores read them)
+    for (int idx = threadIdx.x; idx < NQ * CH; idx += kDecThreads) {
+      const int q = idx / CH, c = idx % CH;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (q < n_rows) {
+        const int r = row0 + q;
+        const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
+        if (r - qh * a.qcap < nq_b) v = *reinterpret_cast<const uint4*>(sK + static_cast<size_t>(r) * (D * 2) + c * 16);
+      }
+      *reinterpret_cast<uint4*>(sQ + sw128_offset(q, c, NQ)) = v;
     }
     __syncthreads();
     if (threadIdx.x < D) {
@@ -411,19 +639,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     if (cs > 1) cluster_sync();   // every CTA holds all nb keys
     else __syncthreads();
-    int* s_wide = reinterpret_cast<int*>(sK + 4096);          // 11-bit first-pass histogram
-    static_assert((RG + 1) * D * 4 <= 4096, "qbar partials overlap the top-C histogram");
+    int* s_wide = reinterpret_cast<int*>(sK + 4096);          // 11-bit first-pass histogram (over the staged rows)
     if (a.nb <= 2 * kDecThreads) cta_topk_linear(s_key, a.nb, a.C, bk->blk, a.C, s_wide, bk->tk);
     else dec_top_c_large(s_key, a.nb, a.C, bk->blk, bk->tk, s_wide);
     // the K and V rings were written and read through the generic proxy above; the
     // producer's TMA writes them next
     fence_proxy_async_smem();
     __syncthreads();
-    if (rank == 0 && a.blocks_out)
+    if (rank == 0 && row0 == 0 && a.blocks_out)
       for (int i = threadIdx.x; i < a.C; i += kDecThreads) a.blocks_out[static_cast<size_t>(bh) * a.C + i] = bk->blk[i];
   }
   if (warp == kDecProducerWarp) {
-    if (!FUSED) init_pipeline();
     if (SPARSE && FUSED) {
       sl_p = fused_block_layout(bk->blk, min(a.C, a.nb), a.S, a.P, a.bs, a.gen_pad, a.box_rows, a.pad_div,
                                 kDecMaxBlocks, kDecMaxSinks, &bk->sl);
@@ -464,20 +690,17 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (deferred) finish_deferred(deferred);
     if (!FUSED && cs > 1) cluster_wait();   // the claim counter is initialised
   }
-  if (warp == kDecMmaWarp) {
-    tmem_alloc(&bk->tmem_base, SM::kTmemCols);
-    tmem_relinquish();
-  }
   if (warp != kDecProducerWarp) {
     // Q rows (query q <-> head kvh*g + q/qcap, position q%qcap) as a K-major SW128 B
     // operand; rows are loaded before the valid count is known and masked afterwards
     const int qt = warp < kDecProducerWarp ? threadIdx.x : threadIdx.x - 32;   // dense index without the producer
-    for (int idx = qt; idx < NQ * CH; idx += kDecThreads - 32) {
+    for (int idx = qt; !FUSED && idx < NQ * CH; idx += kDecThreads - 32) {   // (fused: staged in the prologue)
       const int q = idx / CH, c = idx % CH;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (q < n_rows) {
-        const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
-        const int hq = kvh * a.g + qh, i = q - qh * a.qcap;
+        const int r = row0 + q;
+        const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
+        const int hq = kvh * a.g + qh, i = r - qh * a.qcap;
         v = __ldg(reinterpret_cast<const uint4*>(a.Q + ((static_cast<size_t>(b) * a.Hq + hq) * a.qcap + i) * D) + c);
         if (i >= nq_b) v = make_uint4(0u, 0u, 0u, 0u);
       }
@@ -489,8 +712,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     if (warp < 2) {
       const int q = threadIdx.x;
-      const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
-      const unsigned m = __ballot_sync(0xffffffffu, q < NQ && q < n_rows && (q - qh * a.qcap) < nq_b);
+      const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(row0 + q)));
+      const unsigned m = __ballot_sync(0xffffffffu, q < NQ && q < n_rows && (row0 + q - qh * a.qcap) < nq_b);
       if (lane == 0) bk->qvalid[warp] = m;
     }
     fence_proxy_async_smem();
@@ -796,7 +1019,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   tc_fence_before();
   if (cs > 1) cluster_sync();        // every partial of the cluster is in place
   else __syncthreads();
-  if (warp == kDecMmaWarp) {
+  if (!COLSUM && warp == kDecMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, SM::kTmemCols);
   }
@@ -818,17 +1041,44 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       }
     }
   };
-  auto finish_q = [&](int q, const float4 (&ov)[8], const float2 (&ml)[8]) {
-    float M = -INFINITY;
+  // merged maximum M and row sum l of a query from the CTAs' (m, l); w[r] = 2^(m_r - M)
+  auto merge_ml = [&](const float2 (&ml)[8], float& M, float& l, float (&w)[8]) {
+    M = -INFINITY;
 #pragma unroll
     for (int r = 0; r < 8; ++r)
       if (ml[r].y > 0.f) M = fmaxf(M, ml[r].x);
-    float l = 0.f, w[8];
+    l = 0.f;
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       w[r] = ml[r].y > 0.f ? exp2_approx(ml[r].x - M) : 0.f;
       l += w[r] * ml[r].y;
     }
+  };
+  if constexpr (COLSUM) {
+    // every CTA needs the log-sum-exp of every query column for its column sums
+    if (threadIdx.x < NQ) {
+      const int q = threadIdx.x;
+      float v = INFINITY;                     // not a query: 2^(s - inf) = 0
+      if (q < n_rows) {
+        const int r = row0 + q;
+        const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
+        if (r - qh * a.qcap < nq_b) {
+          float2 ml[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            ml[c] = c < cs ? dsmem_ld_v2(dsmem_addr(smem_u32(part_ml) + static_cast<uint32_t>(q) * 8u, c))
+                           : make_float2(-INFINITY, 0.f);
+          float M, l, w[8];
+          merge_ml(ml, M, l, w);
+          if (l > 0.f) v = M + __log2f(l);
+        }
+      }
+      bk->lse2[q] = v;
+    }
+  }
+  auto finish_q = [&](int q, const float4 (&ov)[8], const float2 (&ml)[8]) {
+    float M, l, w[8];
+    merge_ml(ml, M, l, w);
     const float inv = l > 0.f ? 1.f / l : 0.f;
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -839,8 +1089,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       o.z += wr * ov[r].z;
       o.w += wr * ov[r].w;
     }
-    const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(q)));
-    const int hq = kvh * a.g + qh, i = q - qh * a.qcap;
+    const int r = row0 + q;
+    const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
+    const int hq = kvh * a.g + qh, i = r - qh * a.qcap;
     if (i >= nq_b) o = make_float4(0.f, 0.f, 0.f, 0.f);
     uint2 pk;
     pk.x = pack_bf16x2(o.x, o.y);
@@ -862,9 +1113,23 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (vb) finish_q(qb, ovb, mlb);
     }
   }
-  if (cs > 1) {
-    cluster_arrive_relaxed();        // this warp's reads of the partials are done
-    cluster_wait();                  // no CTA leaves while its partials may still be read
+  if (cs > 1) cluster_arrive_relaxed();   // this warp's reads of the partials are done
+  if constexpr (COLSUM) decode_colsum_phase<NQ, STAGES>(&tmK, a, bk, sK, sV, sQ, tmem, bh);
+  if (cs > 1) cluster_wait();             // no CTA leaves while its partials may still be read
+  if constexpr (COLSUM) {
+    // the column sums are visible to the whole cluster, and no CTA leaves while another
+    // may still claim a tile from CTA 0's counter
+    __threadfence();
+    tc_fence_before();
+    if (cs > 1) cluster_sync();
+    else __syncthreads();
+    if (warp == kDecMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, SM::kTmemCols);
+    }
+    // every CTA of the cluster takes the same barriers here, also after a wait ran out (the
+    // sinks are then undefined, and the device error word says so)
+    if (a.sinks_out) decode_sink_topk(a, bk, sK, bh, rank, cs);
   }
 }
 
@@ -904,7 +1169,7 @@ int dec_make_map(CUtensorMap* map, const void* base, int BH, int L, int box_rows
   return FOCUS_OK;
 }
 
-template <int NQ, int STAGES, bool SPARSE, bool FUSED>
+template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM>
 int max_active_clusters(int cs) {
   static std::mutex mu;
   static std::map<std::pair<int, int>, int> cache;
@@ -914,7 +1179,7 @@ int max_active_clusters(int cs) {
   auto key = std::make_pair(dev, cs);
   auto it = cache.find(key);
   if (it != cache.end()) return it->second;
-  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED>;
+  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED, COLSUM>;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(DecSmem<NQ, STAGES>::kBytes)) !=
       cudaSuccess) {
     cudaGetLastError();
@@ -940,18 +1205,29 @@ int max_active_clusters(int cs) {
   return n;
 }
 
-template <int NQ, int STAGES, bool SPARSE, bool FUSED>
+template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM>
 int choose_cluster(int units) {
   const int sms = device_sm_count();
   for (int cs : {8, 4, 2}) {
     if (units * cs > sms) continue;
-    if (max_active_clusters<NQ, STAGES, SPARSE, FUSED>(cs) >= units) return cs;
+    if (max_active_clusters<NQ, STAGES, SPARSE, FUSED, COLSUM>(cs) >= units) return cs;
   }
   return 1;
 }
 
-template <int NQ, int STAGES, bool SPARSE, bool FUSED>
-int run_decode(const DecArgs& a0, cudaStream_t stream) {
+// Whether the cluster's fused top-S serves S sinks over L columns with cs CTAs; sets the
+// per-CTA share (a multiple of 4 columns) and the columns per thread.
+bool plan_sink_topk(int L, int S, int cs, int* chunk, int* kpt) {
+  const int c = ((L + cs - 1) / cs + 3) & ~3;
+  if (S < 1 || S > kDecMaxSinks || cs * S > 4 * kDecThreads || c > 32 * kDecThreads) return false;
+  if (L - (cs - 1) * c < S) return false;          // the last share holds at least S columns
+  *chunk = c;
+  *kpt = c <= 8 * kDecThreads ? 8 : (c <= 16 * kDecThreads ? 16 : 32);
+  return true;
+}
+
+template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM = false>
+int run_decode(const DecArgs& a0, cudaStream_t stream, bool* sinks_done = nullptr) {
   DecArgs a = a0;
   CUtensorMap mk, mv;
   int st = dec_make_map(&mk, a.K, a.B * a.Hkv, a.L, a.box_rows);
@@ -959,9 +1235,18 @@ int run_decode(const DecArgs& a0, cudaStream_t stream) {
   st = dec_make_map(&mv, a.V, a.B * a.Hkv, a.L, a.box_rows);
   if (st != FOCUS_OK) return st;
   a.dev_err = device_error_word();
-  const int units = a.B * a.Hkv;
-  const int cs = choose_cluster<NQ, STAGES, SPARSE, FUSED>(units);
-  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED>;
+  a.n_slices = (a.g * a.qcap + NQ - 1) / NQ;
+  const int units = a.B * a.Hkv * a.n_slices;
+  if (units > 65535) {
+    set_error("decode attention: %d (sequence, KV head, row slice) units exceed the grid", units);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
+  const int cs = choose_cluster<NQ, STAGES, SPARSE, FUSED, COLSUM>(units);
+  if (COLSUM && a.sinks_out) {
+    if (!plan_sink_topk(a.L, a.S_out, cs, &a.ts_chunk, &a.ts_kpt)) a.sinks_out = nullptr;
+    if (sinks_done) *sinks_done = a.sinks_out != nullptr;
+  }
+  auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED, COLSUM>;
   if (const int st_attr = configure_dynamic_smem(reinterpret_cast<const void*>(kern),
                                                  static_cast<int>(DecSmem<NQ, STAGES>::kBytes),
                                                  "decode attention"))
@@ -984,20 +1269,26 @@ int pow2_divisor(int x, int cap) {
 
 }  // namespace
 
-// Whether the decode kernel serves this shape (else the 128-row tile kernel does).
-bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C) {
-  return d == kDecD && (Hq / Hkv) * qcap <= 64 && L >= 8 && S <= kDecMaxSinks && C <= kDecMaxBlocks;
+// Whether the decode kernel serves this shape (else the 128-row tile kernel does). A sparse
+// call takes up to kDecMaxRows query rows per KV group, in slices of 64 rows that stream
+// the same (few) kept keys. A dense call takes at most one slice: every slice would stream
+// all L keys through a 2-deep ring, and the tile kernel, which reads the keys once per 128
+// rows with every SM busy, does better there.
+bool decode_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C, bool sparse) {
+  const int rows = (Hq / Hkv) * qcap;
+  return d == kDecD && rows <= (sparse ? kDecMaxRows : 64) && L >= 8 && S <= kDecMaxSinks && C <= kDecMaxBlocks;
 }
 
 // Fused relevance + top-C is used when kbar is given (blocks is then ignored).
 bool decode_fused_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C, int nb) {
-  return decode_supported(d, Hq, Hkv, qcap, L, S, C) && nb >= 1 && nb <= kDecMaxNb;
+  return decode_supported(d, Hq, Hkv, qcap, L, S, C, true) && nb >= 1 && nb <= kDecMaxNb;
 }
 
 int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                      __nv_bfloat16* O, float* lse_out, const int32_t* sinks, const int32_t* blocks, int S, int C, int bs,
                      int P, int g0, int g1, bool sparse, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
-                     cudaStream_t stream, const float* kbar, int nb, int32_t* blocks_out) {
+                     cudaStream_t stream, const float* kbar, int nb, int32_t* blocks_out, float* colsum,
+                     int32_t* sinks_out, int S_out, bool* sinks_done) {
   DecArgs a{};
   a.Q = Q;
   a.n_q = n_q;
@@ -1036,7 +1327,7 @@ int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bflo
                             (std::min(S, kDecMaxSinks) + a.box_rows - 1) / a.box_rows * a.box_rows + 256;
     a.pad_div.init(static_cast<uint32_t>(pad_bs), static_cast<uint32_t>(std::min<long long>(n_max, 0xFFFFFFFFll)));
     a.bs_div.init(static_cast<uint32_t>(std::max(bs, 1)), static_cast<uint32_t>(L));
-    a.qcap_div.init(static_cast<uint32_t>(qcap), 64u);
+    a.qcap_div.init(static_cast<uint32_t>(qcap), static_cast<uint32_t>(a.g * qcap));
   }
   const int nrows = a.g * qcap;
   if (kbar) {
@@ -1044,6 +1335,15 @@ int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bflo
     a.nb = nb;
     a.blocks_out = blocks_out;
     return nrows <= 32 ? run_decode<32, 3, true, true>(a, stream) : run_decode<64, 2, true, true>(a, stream);
+  }
+  if (sinks_done) *sinks_done = false;
+  if (!sparse && colsum) {
+    // the sink layer: attention, column sums and (when the cluster can select them) sinks
+    a.colsum = colsum;
+    a.sinks_out = sinks_out;
+    a.S_out = S_out;
+    return nrows <= 32 ? run_decode<32, 3, false, false, true>(a, stream, sinks_done)
+                       : run_decode<64, 2, false, false, true>(a, stream, sinks_done);
   }
   if (nrows <= 32)
     return sparse ? run_decode<32, 3, true, false>(a, stream) : run_decode<32, 3, false, false>(a, stream);

@@ -225,6 +225,12 @@ __device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
       : "memory");
 }
+// L2 prefetch of `bytes` (a multiple of 16; address 16-byte aligned) of global memory: a
+// cache hint with no completion to wait for and no effect on what later loads return.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // L2 policy: lines fetched under it are the first to be evicted (streamed K/V).
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t p;

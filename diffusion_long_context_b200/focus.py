@@ -42,6 +42,7 @@ _SIGS = {
     "focus_block_select": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p]),
     "focus_dense_attention": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "focus_dense_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "focus_dense_attention_sinks": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _i, _p, _p, _sz, _p]),
     "focus_sink_identify": (_i, [_p, _i, _i, _i, _i, _p, _p]),
     "focus_sparse_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                     _p, _p, _sz, _p]),
@@ -207,6 +208,27 @@ def focus_dense_attention(Q, n_q, K, V, O, scale=None, colsum=None, ws=None, str
     st = lib.focus_dense_attention(_ptr(Q), _ptr(n_q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, qcap, float(scale),
                                    _ptr(O), _ptr(colsum), _ptr(ws), ws_bytes, _stream(stream))
     _check(st, "focus_dense_attention")
+
+
+def focus_dense_attention_sinks(Q, n_q, K, V, O, colsum, sinks, scale=None, ws=None, stream=None):
+    """The sink layer: dense attention, column sums and the top-S sinks (S = sinks.shape[2])."""
+    _need(Q, torch.bfloat16, "Q", 4)
+    _need(K, torch.bfloat16, "K", 4)
+    _need(V, torch.bfloat16, "V", 4)
+    _need(O, torch.bfloat16, "O", 4)
+    _need(colsum, torch.float32, "colsum", 3)
+    _need(sinks, torch.int32, "sinks", 3)
+    if n_q is not None:
+        _need(n_q, torch.int32, "n_q", 1)
+    B, Hq, qcap, d = Q.shape
+    Hkv, L = K.shape[1], K.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = dense_workspace_bytes(B, Hq, Hkv, L, d, qcap, True)
+    ws, ws_bytes = _workspace(need, Q.device, ws)
+    st = lib.focus_dense_attention_sinks(_ptr(Q), _ptr(n_q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, qcap, float(scale),
+                                         _ptr(O), _ptr(colsum), sinks.shape[2], _ptr(sinks), _ptr(ws), ws_bytes,
+                                         _stream(stream))
+    _check(st, "focus_dense_attention_sinks")
 
 
 def focus_sink_identify(colsum, S, sinks, stream=None):

@@ -101,11 +101,14 @@ class SparseStep:
         c = self.cfg
         sink_layer = l == c.l_dense
         probs = sink_layer and c.sink_agg == "probs"
-        F.focus_dense_attention(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.O_active[l],
-                                scale=self.scale, colsum=self.colsum if probs else None, ws=self.ws)
         if probs:
-            F.focus_sink_identify(self.colsum, c.S, self.sinks)
-        elif sink_layer:
+            # attention, column sums and the top-S sinks in one call (one launch where served)
+            F.focus_dense_attention_sinks(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.O_active[l],
+                                          self.colsum, self.sinks, scale=self.scale, ws=self.ws)
+            return
+        F.focus_dense_attention(self.Q_active[l], self.n_active, self.K[l], self.V[l], self.O_active[l],
+                                scale=self.scale, ws=self.ws)
+        if sink_layer:
             # mean-query importance: top-S of qbar . k_j over all L keys (each key a block of one)
             F.focus_block_means(self.K[l], c.L, 1, self.k_rows)
             F.focus_block_select(self.Q_active[l], self.n_active, self.k_rows, c.S, self.sinks)

@@ -160,6 +160,22 @@ FOCUS_API int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, con
 FOCUS_API size_t focus_dense_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int qcap, int want_colsum);
 
 /*
+ * (3) The sink layer in one call -- method steps (3) and core method: dense attention of the
+ * active queries (as focus_dense_attention), the sink importance colsum [B, Hkv, L] (as its
+ * colsum_opt) and the sinks [B, Hkv, S] = top-min(S, L) columns of colsum per KV head,
+ * ascending, -1 tail (as focus_sink_identify). Where the few-query kernel serves the shape
+ * (d = 128, (Hq/Hkv) * qcap <= 64) the three run in one launch: after the cluster merge the
+ * kernel re-reads its K tiles, most recent first, for the column sums and selects the sinks
+ * within the cluster; other shapes run the calls in sequence (colsum and sinks are then
+ * still both written). colsum and sinks are required. Requires 1 <= S <= 4096 and the
+ * conditions of focus_dense_attention with column sums; ws/ws_bytes as there.
+ */
+FOCUS_API int focus_dense_attention_sinks(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K,
+                                          const focus_bf16* V, int B, int Hq, int Hkv, int L, int d, int qcap,
+                                          float scale, focus_bf16* O, float* colsum, int S, int32_t* sinks, void* ws,
+                                          size_t ws_bytes, void* stream);
+
+/*
  * (3) Sink identification -- core method / method steps (3): the attention distribution
  * of the sink layer, aggregated over the active queries, picks the S sinks per KV head,
  * reused by every deeper sparse layer. sinks[b, h, :] = top-min(S, L) of colsum[b, h, :],
@@ -189,7 +205,7 @@ FOCUS_API int focus_sparse_attention(const focus_bf16* Q_active, const int32_t* 
  * method steps (4) and (5). Same results as focus_block_select (kept blocks written to
  * blocks [B, Hkv, C], -1 tail) followed by focus_sparse_attention on them. kbar
  * [B, Hkv, nb, d] fp32 with nb = ceil(P / bs). Shapes outside the fused kernel's range
- * (d != 128, more than 64 query rows per KV head, nb > 4096, C > 512 or S > 512) run the
+ * (d != 128, more than 256 query rows per KV head, nb > 4096, C > 512 or S > 512) run the
  * two calls in sequence; ws/ws_bytes then serve focus_sparse_attention (size them with
  * focus_sparse_workspace_bytes).
  */

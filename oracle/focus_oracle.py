@@ -295,14 +295,17 @@ def sparse_step(layer_fn: Callable[[int], Tuple[np.ndarray, np.ndarray, np.ndarr
                 n_layers: int, l_dense: int, conf_prev: np.ndarray, mask: np.ndarray,
                 g0: int, g1: int, n_t: int, rho: float, w: int, P: int, bs: int,
                 C: int, S: int, acap: int, scale: float, layers_out=None, dense_tail: int = 0,
-                relevance: str = "active", sink_agg: str = "probs"):
+                relevance: str = "active", sink_agg: str = "probs", layers_eval=None):
     """One non-block-entry denoising step (method steps (1)-(5)).
 
     layer_fn(l) -> (Q_full [B,Hq,L,d], K, V) in float64. Layers 0..l_dense are dense over
     the active queries; layer l_dense also yields the sinks; deeper layers select top-C
     blocks from their own block means and attend over sinks U blocks U the current block.
-    Returns a dict with I_focus, I_active, sinks, per-layer blocks and outputs (only for
-    layers in `layers_out`, default all).
+    Returns a dict with I_focus, I_active, sinks (and the sink layer's colsum), per-layer
+    blocks and relevance scores R, and outputs (only for layers in `layers_out`, default all).
+    `layers_eval` (default all) limits which layers are computed at all: layer_fn supplies
+    every layer's inputs, so a layer's results depend only on its own inputs and on the
+    sinks of layer l_dense (always computed); the skipped layers are simply absent.
 
     Variants the pages describe: the last `dense_tail` layers also run dense (Dream keeps
     its last 4 layers dense); relevance="focus" scores the blocks with the I_focus rows
@@ -312,10 +315,13 @@ def sparse_step(layer_fn: Callable[[int], Tuple[np.ndarray, np.ndarray, np.ndarr
     """
     focus, active = select_queries(conf_prev, mask, g0, g1, n_t, rho, w)
     n_active = [a.size for a in active]
-    out = {"I_focus": focus, "I_active": active, "O": {}, "blocks": {}, "sinks": None}
+    out = {"I_focus": focus, "I_active": active, "O": {}, "blocks": {}, "R": {}, "sinks": None}
     want = set(range(n_layers)) if layers_out is None else set(layers_out)
+    run = set(range(n_layers)) if layers_eval is None else set(layers_eval) | {l_dense}
     tail0 = max(l_dense + 1, n_layers - dense_tail)
     for l in range(n_layers):
+        if l not in run:
+            continue
         Q, K, V = layer_fn(l)
         Qa = gather_rows(Q, active, acap)
         if l <= l_dense or l >= tail0:
@@ -331,10 +337,11 @@ def sparse_step(layer_fn: Callable[[int], Tuple[np.ndarray, np.ndarray, np.ndarr
             kbar = block_means(K, P, bs)
             if relevance == "focus":
                 Qr = gather_rows(Q, focus, g1 - g0)
-                blocks, _ = block_select(Qr, [f.size for f in focus], kbar, C)
+                blocks, R = block_select(Qr, [f.size for f in focus], kbar, C)
             else:
-                blocks, _ = block_select(Qa, n_active, kbar, C)
+                blocks, R = block_select(Qa, n_active, kbar, C)
             out["blocks"][l] = blocks
+            out["R"][l] = R
             O = sparse_attention(Qa, n_active, K, V, out["sinks"], blocks, bs, P, g0, g1, scale)
         if l in want:
             out["O"][l] = O

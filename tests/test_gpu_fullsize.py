@@ -46,10 +46,10 @@ def _run_two_layers(F, cfg):
         F.focus_gather_rows(Qf, i_active, n_active, Qa)
         O = torch.empty_like(Qa)
         if tag == "dense":
+            # the sink layer as the step runs it: attention, column sums and sinks in one call
             colsum = torch.empty((cfg.B, cfg.Hkv, cfg.L), dtype=torch.float32, device=DEV)
-            F.focus_dense_attention(Qa, n_active, K, V, O, colsum=colsum)
             sinks = torch.empty((cfg.B, cfg.Hkv, cfg.S), **i32)
-            F.focus_sink_identify(colsum, cfg.S, sinks)
+            F.focus_dense_attention_sinks(Qa, n_active, K, V, O, colsum, sinks)
             out.update(colsum=colsum, sinks=sinks)
         else:
             kbar = torch.empty((cfg.B, cfg.Hkv, cfg.nb, cfg.d), dtype=torch.float32, device=DEV)
@@ -123,10 +123,64 @@ def test_full_size_sink_and_sparse_layer(F, cfg):
     _check_against_oracle(cfg, *_run_two_layers(F, cfg))
 
 
-@pytest.mark.parametrize("bs,C,rho", [(32, 8, 4.0), (64, 32, 2.0), (128, 128, 8.0)])
-def test_sweep_points_batch4_32k(F, bs, C, rho):
-    cfg = configs.SWEEP_BASE.replace(bs=bs, C=C, rho=rho, n_layers=2, l_dense=0)
+@pytest.mark.parametrize("point", configs.sweep_points(), ids=lambda p: p.name)
+def test_sweep_points_batch4_32k(F, point):
+    """Every sweep point (B = 4 at 32K; block size x C at rho = 4, and rho = 2, 8): the sink
+    layer and one sparse layer in the bench's launch configuration against the oracle."""
+    cfg = point.replace(n_layers=2, l_dense=0)
     _check_against_oracle(cfg, *_run_two_layers(F, cfg))
+
+
+def test_full_32k_step_as_the_bench_replays_it(F):
+    """The 32-layer 32K step as the bench times it (SparseStep captured in one CUDA graph,
+    fused sparse layers, one-call sink layer), replayed twice, against the oracle's step on
+    the sink layer and sparse layers 3, 17, 20 and 31: I_focus, I_active, the sinks, the kept
+    blocks and the active-query outputs. Layer 20 holds the seeds' one near-tie (KV head 26,
+    relative margin 5.5e-6): a flip there must stay within the tie, and the layer's output is
+    then checked against the oracle run on the GPU's set."""
+    from diffusion_long_context_b200.step import SparseStep
+    cfg = configs.FULL_32K
+    check = [3, 17, 20, 31]
+    st = inputs.step_state(cfg)
+    Q_full = torch.empty((cfg.n_layers, cfg.B, cfg.Hq, cfg.L, cfg.d), dtype=torch.bfloat16, device=DEV)
+    K, V = [], []
+    for l in range(cfg.n_layers):
+        q, k, v = inputs.make_layer(cfg, l, DEV, st.sink_pos)
+        Q_full[l].copy_(q)
+        K.append(k)
+        V.append(v)
+        del q
+    step = SparseStep(cfg, Q_full, K, V, device=DEV, fused=True)
+    step.set_state(torch.from_numpy(st.conf_prev), torch.from_numpy(st.mask), non_blocking=False)
+    step.block_entry()
+    step.capture()
+    step.replay()
+    step.replay()
+    torch.cuda.synchronize()
+    assert F.device_error() == 0
+    rho = float(np.float32(cfg.rho))
+    scale = float(np.float32(1 / math.sqrt(cfg.d)))
+
+    def layer_fn(l):
+        return inputs.to_f64(Q_full[l]), inputs.to_f64(K[l]), inputs.to_f64(V[l])
+
+    ref = orc.sparse_step(layer_fn, cfg.n_layers, cfg.l_dense, st.conf_prev, st.mask, cfg.g0, cfg.g1, cfg.n_t, rho,
+                          cfg.w, cfg.P, cfg.bs, cfg.C, cfg.S, cfg.acap, scale, layers_out=check, layers_eval=check)
+    assert idx_rows(step.i_focus) == [f.tolist() for f in ref["I_focus"]]
+    assert idx_rows(step.i_active) == [a.tolist() for a in ref["I_active"]]
+    nA = [a.size for a in ref["I_active"]]
+    assert assert_index_sets(step.sinks, ref["colsum"], cfg.S, "32K step sinks") == 0
+    for l in check:
+        ties = assert_index_sets(step.blocks[l], ref["R"][l], cfg.C, f"32K step layer {l} blocks")
+        O_ref = ref["O"][l]
+        if ties:
+            assert l == 20, f"layer {l}: unexpected near-tie"
+            Qf, Kl, Vl = layer_fn(l)
+            O_ref = orc.sparse_attention(orc.gather_rows(Qf, ref["I_active"], cfg.acap), nA, Kl, Vl, ref["sinks"],
+                                         step.blocks[l].cpu().numpy().astype(np.int64), cfg.bs, cfg.P, cfg.g0,
+                                         cfg.g1, scale)
+        assert_attention_close(step.O_active[l], O_ref, rows_valid=nA, what=f"32K step layer {l}")
+    step.release()
 
 
 def test_full_refresh_32k_sampled_rows(F):
@@ -147,3 +201,19 @@ def test_full_refresh_32k_sampled_rows(F):
         ref, _, _ = orc.dense_attention(q, None, inputs.to_f64(K[:, hq:hq + 1]), inputs.to_f64(V[:, hq:hq + 1]),
                                         scale)
         assert_attention_close(O[:, hq:hq + 1, ridx], ref, what=f"refresh head {hq}")
+
+
+def test_margin_report_matches_the_generated_inputs():
+    """The recorded top-k margins (tests/golden/topk_margins.txt) were computed on the inputs
+    this device generates: recompute the tiny and 8K rows with the oracle and compare."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.join(os.path.dirname(__file__), "golden"))
+    import make_topk_margins as mk
+    from conftest import GOLDEN
+    with open(os.path.join(GOLDEN, "topk_margins.txt")) as f:
+        recorded = {tuple(ln.split()[:2]): ln.split()[2:] for ln in f if ln.strip() and not ln.startswith("#")}
+    for cfg in (configs.TINY, configs.LLADA_8K):
+        for name, n, k, m, w in mk.margins(cfg, DEV):
+            got = [f"n={n}", f"k={k}", f"min_rel_margin={m:.6e}", f"at={w}"]
+            assert recorded[(cfg.name, name)] == got, (cfg.name, name, got)

@@ -12,8 +12,8 @@ import torch
 
 from diffusion_long_context_b200 import configs, inputs
 from oracle import focus_oracle as orc
-from parity_utils import (KBAR_REL, assert_attention_close, assert_tail_is_minus_one, idx_rows,
-                          topk_matches)
+from parity_utils import (KBAR_REL, assert_attention_close, assert_index_sets, assert_tail_is_minus_one,
+                          idx_rows, topk_matches)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -218,6 +218,9 @@ DENSE_CASES = [
     (1, 2, 1, 129, 128, 16, [16]),
     (1, 8, 4, 700, 128, 32, [27]),          # 2 query heads per KV head x 32: 64 query columns
     (2, 32, 32, 600, 128, 32, [32, 19]),    # 64 heads: clusters of 2
+    (1, 6, 2, 900, 128, 32, [30]),          # 96 rows per KV head: row slices of 64 + 32
+    (2, 28, 4, 1100, 128, 24, [24, 7]),     # GQA 7:1, 168 rows per KV head: three row slices
+    (1, 16, 1, 700, 128, 32, [32]),         # 512 rows per KV head: the 128-row tile kernel
 ]
 
 
@@ -228,14 +231,17 @@ def test_dense_attention_active_with_colsum(F, B, Hq, Hkv, L, d, qcap, n_q):
     V = inputs.random_bf16((B, Hkv, L, d), seed=L + 2, device=DEV)
     nq = torch.tensor(n_q, dtype=torch.int32, device=DEV)
     O = torch.full((B, Hq, qcap, d), 7.0, dtype=torch.bfloat16, device=DEV)
-    colsum = torch.empty((B, Hkv, L), dtype=torch.float32, device=DEV)
+    # column sums are served for up to 256 query rows per KV group
+    want_colsum = (Hq // Hkv) * qcap <= 256
+    colsum = torch.empty((B, Hkv, L), dtype=torch.float32, device=DEV) if want_colsum else None
     scale = 1.0 / math.sqrt(d)
     F.focus_dense_attention(Q, nq, K, V, O, scale=scale, colsum=colsum)
     torch.cuda.synchronize()
     refO, refC, _ = orc.dense_attention(inputs.to_f64(Q), n_q, inputs.to_f64(K), inputs.to_f64(V),
                                         float(np.float32(scale)), want_colsum=True)
     assert_attention_close(O, refO, rows_valid=n_q, what="dense attention")
-    np.testing.assert_allclose(colsum.cpu().double().numpy(), refC, rtol=2e-3, atol=1e-6)
+    if want_colsum:
+        np.testing.assert_allclose(colsum.cpu().double().numpy(), refC, rtol=2e-3, atol=1e-6)
     assert F.device_error() == 0
 
 
@@ -250,6 +256,66 @@ def test_dense_attention_full_refresh(F, B, Hq, Hkv, L, d):
     refO, _, _ = orc.dense_attention(inputs.to_f64(Q), None, inputs.to_f64(K), inputs.to_f64(V),
                                      float(np.float32(1.0 / math.sqrt(d))))
     assert_attention_close(O, refO, what="full refresh")
+
+
+SINK_LAYER_CASES = [
+    # B, Hq, Hkv, L, d, qcap, n_q, S
+    (1, 32, 32, 4000, 128, 32, [30], 32),     # one launch: attention, column sums, cluster top-S
+    (2, 4, 4, 2500, 128, 32, [32, 7], 16),    # clusters of 8 CTAs
+    (1, 8, 4, 1200, 128, 32, [27], 8),        # 64 rows per KV head: the 64-column kernel
+    (1, 2, 1, 129, 128, 16, [16], 4),         # one partial key tile
+    (1, 4, 4, 300, 128, 32, [31], 120),       # the last share holds fewer than S columns: top-S kernel
+    (1, 2, 2, 5000, 128, 32, [32], 700),      # S beyond the cluster's candidate room: top-S kernel
+    (1, 4, 4, 700, 64, 32, [25], 8),          # d = 64: tile kernel, column-sum kernel, top-S kernel
+    (1, 28, 4, 900, 128, 32, [29], 16),       # 224 rows per KV head: tile kernel + column-sum kernel
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,d,qcap,n_q,S", SINK_LAYER_CASES)
+def test_sink_layer_one_call(F, B, Hq, Hkv, L, d, qcap, n_q, S):
+    """focus_dense_attention_sinks against the oracle: output rows, column sums, and the
+    top-S sets (bit-exact up to near-ties at the boundary)."""
+    Q = inputs.random_bf16((B, Hq, qcap, d), seed=5 * L + S, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=5 * L + S + 1, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=5 * L + S + 2, device=DEV)
+    nq = torch.tensor(n_q, dtype=torch.int32, device=DEV)
+    O = torch.full((B, Hq, qcap, d), 3.0, dtype=torch.bfloat16, device=DEV)
+    colsum = torch.full((B, Hkv, L), -1.0, dtype=torch.float32, device=DEV)
+    sinks = torch.full((B, Hkv, S), -7, dtype=torch.int32, device=DEV)
+    scale = 1.0 / math.sqrt(d)
+    F.focus_dense_attention_sinks(Q, nq, K, V, O, colsum, sinks, scale=scale)
+    torch.cuda.synchronize()
+    assert F.device_error() == 0
+    refO, refC, _ = orc.dense_attention(inputs.to_f64(Q), n_q, inputs.to_f64(K), inputs.to_f64(V),
+                                        float(np.float32(scale)), want_colsum=True)
+    assert_attention_close(O, refO, rows_valid=n_q, what="sink layer attention")
+    np.testing.assert_allclose(colsum.cpu().double().numpy(), refC, rtol=2e-3, atol=1e-6)
+    ties = assert_index_sets(sinks, refC, min(S, L), "sink layer sinks")
+    assert ties == 0, f"{ties} near-tie sink sets"
+
+
+def test_sink_layer_cluster_top_s_matches_the_top_s_kernel(F):
+    """On the 32K step's shape (reduced length) the one-call sink layer's in-cluster top-S
+    picks the sets focus_sink_identify picks from the column sums of focus_dense_attention
+    (the same kernel; its CTAs claim key tiles dynamically, so the order of the fp32 partial
+    sums, and with it the last bits of O and of the column sums, varies between launches)."""
+    B, Hq, Hkv, L, d, qcap, S = 1, 32, 32, 12288, 128, 32, 32
+    Q = inputs.random_bf16((B, Hq, qcap, d), seed=901, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=902, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=903, device=DEV)
+    nq = torch.tensor([30], dtype=torch.int32, device=DEV)
+    O1, O2 = (torch.empty((B, Hq, qcap, d), dtype=torch.bfloat16, device=DEV) for _ in range(2))
+    c1, c2 = (torch.empty((B, Hkv, L), dtype=torch.float32, device=DEV) for _ in range(2))
+    s1, s2 = (torch.empty((B, Hkv, S), dtype=torch.int32, device=DEV) for _ in range(2))
+    F.focus_dense_attention_sinks(Q, nq, K, V, O1, c1, s1)
+    F.focus_dense_attention(Q, nq, K, V, O2, colsum=c2)
+    F.focus_sink_identify(c2, S, s2)
+    torch.cuda.synchronize()
+    assert F.device_error() == 0
+    torch.testing.assert_close(O1.float(), O2.float(), rtol=0, atol=2e-3)
+    torch.testing.assert_close(c1, c2, rtol=1e-5, atol=0)
+    assert assert_index_sets(s1, c2.double().cpu().numpy(), S, "one-call sinks vs the top-S kernel") == 0
+    assert assert_index_sets(s2, c1.double().cpu().numpy(), S, "top-S kernel vs one-call column sums") == 0
 
 
 def test_dense_attention_planted_sinks_recovered(F):
@@ -289,6 +355,8 @@ SPARSE_CASES = [
     ("gqa2_nq64", 1, 8, 4, 128, 1024, 32, 1100, 64, 5, 9, 32, [32]),
     ("mha64_heads", 2, 32, 32, 128, 640, 32, 700, 32, 4, 6, 32, [25, 32]),
     ("bs16_mha", 1, 4, 4, 128, 512, 32, 560, 16, 12, 5, 32, [30]),
+    ("gqa3_96rows", 2, 6, 2, 128, 1024, 32, 1100, 64, 7, 5, 32, [32, 12]),
+    ("gqa16_tile", 1, 16, 1, 128, 1024, 32, 1088, 64, 6, 4, 32, [29]),
 ]
 
 
@@ -412,7 +480,9 @@ FUSED_CASES = [
     ("mha_b2_bs32", 2, 4, 4, 1024, 32, 1088, 32, 12, 16, 32, [32, 9]),
     ("gqa2", 1, 8, 4, 1500, 32, 1600, 64, 5, 6, 32, [27]),
     ("ragged_bs24", 1, 2, 2, 250, 20, 300, 24, 4, 3, 20, [20]),
-    ("gqa7_fallback", 1, 28, 4, 1024, 32, 1100, 64, 6, 8, 32, [31]),     # 224 rows: two-call path
+    ("gqa7_sliced", 1, 28, 4, 1024, 32, 1100, 64, 6, 8, 32, [31]),       # 224 rows: four row slices
+    ("gqa3_b2", 2, 6, 2, 1024, 32, 1100, 64, 7, 5, 32, [32, 12]),         # 96 rows: two slices
+    ("gqa16_two_calls", 1, 16, 1, 1024, 32, 1100, 64, 6, 8, 32, [31]),   # 512 rows: two-call path
 ]
 
 

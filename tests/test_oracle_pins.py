@@ -435,3 +435,21 @@ def test_variant_schedules_and_ratio_forms():
     r = cf.ratio_forms(cf.FULL_32K)               # alpha = 0.5 of 508 blocks, 1% of 32768 tokens
     assert (r.C, r.S) == (254, 328)
     assert cf.ratio_forms(cf.TINY).C == 7 and cf.ratio_forms(cf.TINY).S == 6
+
+
+def test_step_layer_subset_equals_the_full_step():
+    """sparse_step(layers_eval=...) computes the chosen layers exactly as the full step does:
+    the layers' inputs come from layer_fn, so only the sinks carry from layer to layer."""
+    from diffusion_long_context_b200 import configs as cf
+    from diffusion_long_context_b200 import inputs as inp
+    cfg = cf.scaled(cf.LLADA_8K, 768, n_layers=5, Hq=4, Hkv=2, l_dense=1, C=3, S=4, bs=32)
+    st = inp.step_state(cfg)
+    lay = [tuple(inp.to_f64(t) for t in inp.make_layer(cfg, l, "cpu", st.sink_pos)) for l in range(cfg.n_layers)]
+    args = (cfg.n_layers, cfg.l_dense, st.conf_prev, st.mask, cfg.g0, cfg.g1, cfg.n_t, cfg.rho, cfg.w, cfg.P, cfg.bs,
+            cfg.C, cfg.S, cfg.acap, 1 / math.sqrt(cfg.d))
+    full = orc.sparse_step(lambda l: lay[l], *args)
+    part = orc.sparse_step(lambda l: lay[l], *args, layers_eval=[3])
+    assert np.array_equal(full["sinks"], part["sinks"])
+    assert sorted(part["blocks"]) == [3] and sorted(part["O"]) == [1, 3]
+    assert np.array_equal(full["blocks"][3], part["blocks"][3]) and np.array_equal(full["R"][3], part["R"][3])
+    assert np.array_equal(full["O"][3], part["O"][3])

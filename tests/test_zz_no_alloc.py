@@ -36,7 +36,7 @@ def _p(t):
     return ctypes.c_void_p(0 if t is None else t.data_ptr())
 
 
-def _case(seed, B=1, Hq=8, Hkv=1, d=128, P=4096, G=32, bs=64, C=32, S=16, acap=32):
+def _case(seed, B=1, Hq=16, Hkv=1, d=128, P=4096, G=32, bs=64, C=32, S=16, acap=32):
     g0, g1 = P, P + G
     L = g1 + 64
     rng = np.random.default_rng(seed)
@@ -63,8 +63,8 @@ def _noalloc(F, c, O, stream):
 
 def test_noalloc_matches_the_workspace_entry_point_twice(F):
     stream = torch.cuda.current_stream()
-    # 8 query heads x 32 queries on one KV head: the 128-row tile kernel with split-KV
-    # partials in the scratch array
+    # 16 query heads x 32 queries on one KV head (512 rows): the 128-row tile kernel with
+    # split-KV partials in the scratch array
     for seed in (11, 12):                                  # two calls in a row, different inputs
         c = _case(seed)
         S, C, bs, P, g0, g1, B, Hq, Hkv, L, d, acap = c["sizes"]
