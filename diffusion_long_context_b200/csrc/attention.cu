@@ -16,9 +16,9 @@
 // Per 128-key tile: S = Q K^T (M=128, N=128, K=d) into TMEM, softmax in registers,
 // P (bf16) to shared memory, O += P V (M=128, N=d, K=128) into TMEM.
 //
-// The sparse key sequence is laid out as slots: each selected block padded to a
-// multiple of 8 slots, then the current block padded to 8, then the de-duplicated
-// sinks. Every 8-slot group of a block or of the current block is a contiguous key run
+// The sparse key sequence is laid out as slots (slots.cuh): the current block, then each
+// kept block padded to a multiple of 8 slots, then the de-duplicated sinks. Every
+// box-aligned group of slots of a block or of the current block is a contiguous key run
 // and is fetched by one TMA box per 64-column atom; sink slots are fetched row by row.
 // Padding slots are masked out of the softmax.
 #include <cuda.h>
@@ -41,6 +41,11 @@ int decode_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bflo
                      float* colsum = nullptr, int32_t* sinks_out = nullptr, int S_out = 0,
                      bool* sinks_done = nullptr);
 bool decode_fused_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int C, int nb);
+// refresh.cu
+bool refresh_supported(int d, int B, int Hq, int Hkv, int qcap, int sms);
+int refresh_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
+                      __nv_bfloat16* O, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
+                      cudaStream_t stream);
 
 constexpr int kBM = 128;            // query rows per CTA (tcgen05 M)
 constexpr int kBN = 128;            // keys per tile
@@ -769,6 +774,7 @@ int gen_pad_for(int box_rows, int G) { return (G + box_rows - 1) / box_rows * bo
 
 struct AttnPlan {
   bool decode;            // few-query swap-AB kernel (decode_attention.cu) serves this call
+  bool refresh;           // many-row kernel (refresh.cu) serves this dense call
   int n_mtiles, n_splits, tiles_per_split;
   size_t lse_bytes, part_lse_bytes, part_o_bytes, total;
 };
@@ -781,6 +787,11 @@ AttnPlan plan_attention(int B, int Hq, int Hkv, int d, int qcap, int kv_cap, boo
   const int g = Hq / Hkv;
   if (decode_supported(d, Hq, Hkv, qcap, L, S, C, sparse)) {
     p.decode = true;                   // merges its splits in the cluster; column sums in-kernel
+    p.n_splits = 1;
+    return p;
+  }
+  if (!sparse && !want_lse && refresh_supported(d, B, Hq, Hkv, qcap, device_sm_count())) {
+    p.refresh = true;                  // every row block streams all keys: no splits, no workspace
     p.n_splits = 1;
     return p;
   }
@@ -894,6 +905,9 @@ int run_attention(AttnArgs args, const AttnPlan& plan, void* ws, float* colsum, 
                   int32_t* sinks_out = nullptr, int S_out = 0, bool* sinks_done = nullptr) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   if (sinks_done) *sinks_done = false;
+  if (plan.refresh)
+    return refresh_attention(args.Q, args.n_q, args.K, args.V, args.O, args.B, args.Hq, args.Hkv, args.L, args.qcap,
+                             args.scale_log2, stream);
   if (plan.decode) {
     // the decode kernel forms the column sums (and, where it can, the sinks) itself
     return decode_attention(args.Q, args.n_q, args.K, args.V, args.O, nullptr, args.sinks, args.blocks, args.S,

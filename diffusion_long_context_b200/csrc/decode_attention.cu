@@ -81,7 +81,7 @@ struct DecArgs {
   int32_t* sinks_out;
   int S_out;
   int ts_chunk;                // columns per CTA for the top-S (a multiple of 4)
-  int ts_kpt;                  // columns per thread for it: 8, 16 or 32
+  int ts_kpt;                  // columns per thread for it (8)
 };
 
 struct __align__(8) DecBook {
@@ -108,7 +108,6 @@ struct __align__(8) DecBook {
   uint64_t c_full[6], c_empty[6], c_sfull[2], c_sfree[2];
   int c_tile[6];           // tile held by each column-sum slot
   int c_stile[2];          // tile whose scores an S buffer holds, -1 = end
-  uint32_t c_ctr;          // tiles claimed so far for the column-sum pass (CTA 0)
   float lse2[64];          // log2-domain log-sum-exp of every query column (+inf: not a query)
 };
 
@@ -151,15 +150,18 @@ __device__ __noinline__ void dec_top_c_large(const uint32_t* s_key, int nb, int 
 // sink layer, aggregated over the active queries, identifies the sinks). They run after
 // the cluster merge, once the log-sum-exp of every query is known:
 //   colsum[b, h, key] = sum over query columns q of 2^(scale_log2 * s[key, q] - lse2[q]).
-// The CTAs claim 128-key tiles from a counter in CTA 0, from the last tile down, so the
-// tiles the attention pass read last (the ones most likely still in L2: the pass loaded K
-// without the evict-first hint it gives V) come first. K tiles flow through a CS-slot ring
+// CTA r takes the 128-key tiles p_n - 1 - r, p_n - 1 - r - cs, ...: from the last tile
+// down (the tiles the attention pass read last first), with no claim round trip on the
+// producer's path. The pass re-reads K from HBM: an evict-last hint on the attention
+// pass's K loads (V evict-first) was measured to leave the column-sum pass at the same
+// 6.1 TB/s, i.e. no reuse out of L2 at this size (268 MB of K at 32K). K tiles flow through a CS-slot ring
 // made of the K ring and the V-ring stages the merge does not read; S^T = K_tile . Q^T
 // lands in the two S buffers of tensor memory; each softmax thread owns one key, the two
 // query halves of a key are added through shared memory, and the key's sum is stored.
 template <int NQ, int STAGES>
 __device__ __noinline__ void decode_colsum_phase(const CUtensorMap* tmK, const DecArgs& a, DecBook* bk, uint8_t* sK,
-                                                 uint8_t* sV, const uint8_t* sQ, uint32_t tmem, int bh) {
+                                                 uint8_t* sV, const uint8_t* sQ, uint32_t tmem, int bh, int rank,
+                                                 int cs) {
   using SM = DecSmem<NQ, STAGES>;
   constexpr int D = kDecD;
   constexpr int QH = NQ / 2;
@@ -179,14 +181,13 @@ __device__ __noinline__ void decode_colsum_phase(const CUtensorMap* tmK, const D
   };
   if (warp == kDecProducerWarp) {
     if (lane == 0) {
-      const uint32_t ctr = smem_u32(&bk->c_ctr);
       const uint64_t l2_once = l2_evict_first_policy();   // the last read of these K rows
       for (int it = 0;; ++it) {
         const int sl = it % CS;
         if (it >= CS && !mbar_wait(&bk->c_empty[sl], ((it / CS) - 1) & 1, abort_flag, a.dev_err,
                                    DEV_ERR_TIMEOUT_PRODUCER))
           break;
-        const int tile = p_n - 1 - static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
+        const int tile = p_n - 1 - (rank + it * cs);
         if (tile < 0) {
           bk->c_tile[sl] = -1;
           mbar_arrive(&bk->c_full[sl]);
@@ -297,9 +298,7 @@ __device__ __noinline__ void decode_sink_topk(const DecArgs& a, DecBook* bk, uin
   int* s_priv = reinterpret_cast<int*>(s_pos + S);                            // per-warp histograms
   int* s_wide = s_priv + 2 * (kDecThreads / 32) * 257;                        // [2048 + 64]
   const float* row = a.colsum + static_cast<size_t>(bh) * a.L + c0;
-  if (a.ts_kpt <= 8) decode_topk_share<8>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);
-  else if (a.ts_kpt <= 16) decode_topk_share<16>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);
-  else decode_topk_share<32>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);
+  decode_topk_share<8>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);   // n <= 8 * threads
   __syncthreads();
   const uint32_t ck0 = smem_u32(s_ckey), ci0 = smem_u32(s_cidx);
   for (int i = threadIdx.x; i < S; i += kDecThreads) {
@@ -406,7 +405,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int at = (j >> 1) & 1;
       const uint32_t off = at * (128 * 128) + grp * BR * 128;
       if (j & 1) tma_load_3d_hint(smem_u32(dV + off), &tmV, &bk->full[s], at * 64, k0, bh, l2_stream);
-      else if (COLSUM) tma_load_3d(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh);   // read again below
       else tma_load_3d_hint(smem_u32(dK + off), &tmK, &bk->full[s], at * 64, k0, bh, l2_stream);
     }
     if (SPARSE && tma_mask != all_groups) {
@@ -494,7 +492,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           mbar_init(&bk->c_sfull[i], 2);      // the MMAs' commit + the tile id published
           mbar_init(&bk->c_sfree[i], kDecSoftmaxWarps);
         }
-        if (rank == 0) bk->c_ctr = 0u;
       }
       bk->abort_flag = 0;
       if (rank == 0) bk->tile_ctr = static_cast<uint32_t>(cs * STAGES);
@@ -525,7 +522,22 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // ---------------------------------------------------------------- prologue
   // The producer warp builds the slot layout and issues the first STAGES tiles before the
-  // CTA barrier; meanwhile the other warps stage Q.
+  // CTA barrier; meanwhile the other warps stage Q. The fused form first stages the group's
+  // query rows (into the idle K ring) and its first round of block means (into the idle V
+  // ring) by bulk copies, issued before anything else.
+  constexpr int kKbRound = STAGES >= 3 ? 128 : 120;            // kbar rows per round
+  if (FUSED && threadIdx.x == 0) {
+    const uint32_t qbytes = static_cast<uint32_t>(a.g * a.qcap * D * 2);
+    mbar_arrive_expect_tx(&bk->q_bar, qbytes);
+    bulk_load(smem_u32(sK), a.Q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * a.g) * a.qcap * D,
+              qbytes, &bk->q_bar);
+    if (j_begin < j_end) {
+      const int nrow = min(kKbRound, j_end - j_begin);
+      mbar_arrive_expect_tx(&bk->kb_bar, static_cast<uint32_t>(nrow * D * 4));
+      bulk_load(smem_u32(sV), kb + static_cast<size_t>(j_begin) * D, static_cast<uint32_t>(nrow * D * 4),
+                &bk->kb_bar);
+    }
+  }
   const int nq_b = a.n_q ? min(a.n_q[b], a.qcap) : a.qcap;
   if (SPARSE && warp == kDecProducerWarp) {
     // kept-block list and sinks of this (b, h): their first entries are fetched right away
@@ -540,10 +552,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // (contiguous in Q) are staged into the (still idle) K ring by one bulk copy issued
     // with the first round, and qbar is summed from there.
     constexpr int RG = kDecThreads / 64;                       // qbar row groups
-    constexpr int kKbRound = STAGES >= 3 ? 128 : 120;          // leaves room for the qbar partials
     static_assert(kKbRound * D * 4 + (RG + 1) * D * 4 <= STAGES * SM::kTile, "kbar round exceeds the V ring");
     static_assert(kDecMaxRows * D * 2 <= STAGES * SM::kTile, "the group's query rows exceed the K ring");
-    const __nv_bfloat162* s_qrows = reinterpret_cast<const __nv_bfloat162*>(sK);   // [g * qcap][D / 2]
+    uint8_t* const sQraw = sK;                                 // [g * qcap][D] bf16
+    const __nv_bfloat162* s_qrows = reinterpret_cast<const __nv_bfloat162*>(sQraw);
     float* s_kb = reinterpret_cast<float*>(sV);                // [kKbRound][D]
     float* s_part = s_kb + kKbRound * D;                       // [RG][D]
     float* s_qbar = s_part + RG * D;                           // [D]
@@ -557,13 +569,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_arrive_expect_tx(&bk->kb_bar, static_cast<uint32_t>(nrow * D * 4));
       bulk_load(smem_u32(s_kb), kb + static_cast<size_t>(j0) * D, static_cast<uint32_t>(nrow * D * 4), &bk->kb_bar);
     };
-    if (threadIdx.x == 0) {
-      const uint32_t qbytes = static_cast<uint32_t>(nr * D * 2);
-      mbar_arrive_expect_tx(&bk->q_bar, qbytes);
-      bulk_load(smem_u32(sK), a.Q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * a.g) * a.qcap * D,
-                qbytes, &bk->q_bar);
-      if (j_begin < j_end) issue_round(j_begin);
-    }
     // qbar over the group's valid rows: RG row groups x 64 dim pairs. Row r is query head
     // r / qcap at position i = r % qcap, valid when i < nq_b.
     {
@@ -593,7 +598,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       if (q < n_rows) {
         const int r = row0 + q;
         const int qh = static_cast<int>(qdiv.div(static_cast<uint32_t>(r)));
-        if (r - qh * a.qcap < nq_b) v = *reinterpret_cast<const uint4*>(sK + static_cast<size_t>(r) * (D * 2) + c * 16);
+        if (r - qh * a.qcap < nq_b) v = *reinterpret_cast<const uint4*>(sQraw + static_cast<size_t>(r) * (D * 2) + c * 16);
       }
       *reinterpret_cast<uint4*>(sQ + sw128_offset(q, c, NQ)) = v;
     }
@@ -639,7 +644,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     if (cs > 1) cluster_sync();   // every CTA holds all nb keys
     else __syncthreads();
-    int* s_wide = reinterpret_cast<int*>(sK + 4096);          // 11-bit first-pass histogram (over the staged rows)
+    int* s_wide = reinterpret_cast<int*>(sK + 4096);          // 11-bit first pass (over the staged rows)
     if (a.nb <= 2 * kDecThreads) cta_topk_linear(s_key, a.nb, a.C, bk->blk, a.C, s_wide, bk->tk);
     else dec_top_c_large(s_key, a.nb, a.C, bk->blk, bk->tk, s_wide);
     // the K and V rings were written and read through the generic proxy above; the
@@ -665,9 +670,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     // the layout and the barriers are ready: release the other warps, then fill the ring
     // (a tile gathered row by row completes after the TMA tiles behind it are issued)
     named_bar_arrive(2, kDecThreads);
-    // Tiles of kept blocks and of the current block do not need the sinks: they are issued
-    // first, and the sinks are de-duplicated just before the first tile that holds sink
-    // slots, at the latest before any tile beyond this first round.
+    // Tiles of kept blocks and of the current block do not need the sinks: the sinks are
+    // de-duplicated just before the first tile that holds sink slots (the sink segment ends
+    // the layout), at the latest before any tile beyond this first round.
     bool sinks_ready = !SPARSE;
     auto ensure_sinks = [&]() {
       if (SPARSE && !sinks_ready) {
@@ -683,7 +688,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         p_more = false;
         break;
       }
-      if (tile * 128 < sl_p.gen_start) ensure_sinks();
+      if ((tile + 1) * 128 > sl_p.sink_start) ensure_sinks();
       if (produce(it, tile, true)) deferred |= 1u << it;
     }
     ensure_sinks();
@@ -744,11 +749,20 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       // trip to CTA 0) is first read after the next stage wait, so it never delays a load.
       // The claimed tile is planned while its stage is still busy (the claim has long
       // returned by then), so a freed stage is refilled at once.
+      // The sparse layout ends with the sink segment, whose rows are gathered one by one:
+      // its last tile is handed out in the middle of the claims (claim m), so that the
+      // gather is issued while the claiming CTA still has other tiles to consume and the
+      // claims after it rebalance the cluster, instead of ending some CTA's work late.
+      const int m_sink = max(cs * STAGES, p_n / 2);
+      auto claim_tile = [&](int c) {
+        if (!SPARSE || m_sink >= p_n - 1 || c < m_sink || c >= p_n) return c;
+        return c == m_sink ? p_n - 1 : c - 1;
+      };
       int claim = 0;
       if (lane == 0) claim = static_cast<int>(dsmem_atomic_add(ctr, 0, 1u));
       for (int it = STAGES;; ++it) {
         const int s = it % STAGES;
-        const int tile = __shfl_sync(0xffffffffu, claim, 0);
+        const int tile = claim_tile(__shfl_sync(0xffffffffu, claim, 0));
         TilePlan pl{0u, 0, 0};
         if (tile < p_n) pl = plan_tile(tile);
         if (!__all_sync(0xffffffffu, mbar_wait(&bk->empty[s], ((it / STAGES) - 1) & 1, abort_flag, a.dev_err,
@@ -1055,9 +1069,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
   };
   if constexpr (COLSUM) {
-    // every CTA needs the log-sum-exp of every query column for its column sums
-    if (threadIdx.x < NQ) {
-      const int q = threadIdx.x;
+    // every CTA needs the log-sum-exp of every query column for its column sums: the
+    // producer warp, idle now, forms it while the softmax warps merge
+    for (int q = lane; warp == kDecProducerWarp && q < NQ; q += 32) {
       float v = INFINITY;                     // not a query: 2^(s - inf) = 0
       if (q < n_rows) {
         const int r = row0 + q;
@@ -1114,11 +1128,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
   }
   if (cs > 1) cluster_arrive_relaxed();   // this warp's reads of the partials are done
-  if constexpr (COLSUM) decode_colsum_phase<NQ, STAGES>(&tmK, a, bk, sK, sV, sQ, tmem, bh);
+  if constexpr (COLSUM) decode_colsum_phase<NQ, STAGES>(&tmK, a, bk, sK, sV, sQ, tmem, bh, rank, cs);
   if (cs > 1) cluster_wait();             // no CTA leaves while its partials may still be read
   if constexpr (COLSUM) {
-    // the column sums are visible to the whole cluster, and no CTA leaves while another
-    // may still claim a tile from CTA 0's counter
+    // the column sums are visible to the whole cluster
     __threadfence();
     tc_fence_before();
     if (cs > 1) cluster_sync();
@@ -1216,13 +1229,17 @@ int choose_cluster(int units) {
 }
 
 // Whether the cluster's fused top-S serves S sinks over L columns with cs CTAs; sets the
-// per-CTA share (a multiple of 4 columns) and the columns per thread.
+// per-CTA share (a multiple of 4 columns) and the columns per thread. The selection's
+// passes cost in proportion to the columns per thread: up to 8 per thread (a 2560-column
+// share) it beats a separate launch (measured at 8K: the sink layer 59 -> 53 us); at
+// 32K's 8192-column shares it took 29 us against about 12 us for the top-S kernel, whose
+// 8-CTA clusters of 512 threads hold 8 columns per thread, so longer rows use that kernel.
 bool plan_sink_topk(int L, int S, int cs, int* chunk, int* kpt) {
   const int c = ((L + cs - 1) / cs + 3) & ~3;
-  if (S < 1 || S > kDecMaxSinks || cs * S > 4 * kDecThreads || c > 32 * kDecThreads) return false;
+  if (S < 1 || S > kDecMaxSinks || cs * S > 4 * kDecThreads || c > 8 * kDecThreads) return false;
   if (L - (cs - 1) * c < S) return false;          // the last share holds at least S columns
   *chunk = c;
-  *kpt = c <= 8 * kDecThreads ? 8 : (c <= 16 * kDecThreads ? 16 : 32);
+  *kpt = 8;
   return true;
 }
 

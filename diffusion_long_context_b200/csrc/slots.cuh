@@ -3,16 +3,17 @@
 // Dense: slot s is key s, s < L.
 // Sparse (Focus-dLLM method steps (5): I_p = sinks U kept prompt blocks U current
 // block, each key once): slots are laid out as
+//   [ current block [g0, g1) ]             padded to gen_pad slots (a multiple of box_rows >= G)
+//   [ kept block 0 | kept block 1 | ... ]  each padded to pad_bs = round_up(bs, 8)
 //   [ sinks ]                              one slot per listed sink; sinks inside a kept
 //                                          block or the current block, out-of-range and
 //                                          repeated entries are dropped (invalid slots);
 //                                          padded to a multiple of box_rows
-//   [ current block [g0, g1) ]             padded to gen_pad slots (a multiple of box_rows >= G)
-//   [ kept block 0 | kept block 1 | ... ]  each padded to pad_bs = round_up(bs, 8)
 // Padding slots are invalid (masked out of the softmax). Every box_rows-aligned group of
 // slots inside the current block or a kept block is one contiguous run of keys and can be
-// fetched by one TMA box; sink slots are fetched row by row. The sinks come first so that
-// their row-by-row gather starts with the first tile instead of ending the key sequence.
+// fetched by one TMA box; sink slots are fetched row by row. The sinks come last: with
+// tiles claimed a ring's depth ahead of their use, the slow row-by-row gather is issued
+// while earlier tiles are still being consumed, instead of holding up the first tile.
 #pragma once
 
 #include "focus_common.cuh"
@@ -21,9 +22,9 @@ namespace focus {
 
 struct SlotLayout {
   int n_slots;      // total slots (keys + padding)
-  int n_sinks;      // sink slots [0, n_sinks), one per listed sink (-1 where dropped)
-  int gen_start;    // first slot of the current block
-  int blk_start;    // first slot of the kept blocks
+  int n_sinks;      // sink slots [sink_start, sink_start + n_sinks), one per listed sink
+  int blk_start;    // first slot of the kept blocks (the current block starts at slot 0)
+  int sink_start;   // first slot of the sinks
   int pad_bs;       // slots per kept block
   int nvb;          // kept blocks (valid entries of the block list)
   int last_size;    // valid keys of the last kept block (short when it ends at P)
@@ -80,9 +81,9 @@ __device__ __forceinline__ SlotLayout build_block_layout(const LayoutPrefetch& p
   sl.nvb = nvb;
   sl.last_size = nvb > 0 ? min(bs, P - s_blk[nvb - 1] * bs) : bs;
   sl.n_sinks = min(S, max_sinks);
-  sl.gen_start = (sl.n_sinks + box_rows - 1) & ~(box_rows - 1);
-  sl.blk_start = sl.gen_start + gen_pad;
-  sl.n_slots = sl.blk_start + nvb * sl.pad_bs;
+  sl.blk_start = gen_pad;
+  sl.sink_start = sl.blk_start + nvb * sl.pad_bs;
+  sl.n_slots = sl.sink_start + ((sl.n_sinks + box_rows - 1) & ~(box_rows - 1));
   sl.pad_div = pad_div;
   if (lane == 0) *out = sl;
   return sl;
@@ -100,18 +101,18 @@ __device__ __forceinline__ SlotLayout fused_block_layout(const int* s_blk, int n
   sl.nvb = nvb;
   sl.last_size = nvb > 0 ? min(bs, P - s_blk[nvb - 1] * bs) : bs;
   sl.n_sinks = min(S, max_sinks);
-  sl.gen_start = (sl.n_sinks + box_rows - 1) & ~(box_rows - 1);
-  sl.blk_start = sl.gen_start + gen_pad;
-  sl.n_slots = sl.blk_start + nvb * sl.pad_bs;
+  sl.blk_start = gen_pad;
+  sl.sink_start = sl.blk_start + nvb * sl.pad_bs;
+  sl.n_slots = sl.sink_start + ((sl.n_sinks + box_rows - 1) & ~(box_rows - 1));
   sl.pad_div = pad_div;
   if (lane == 0) *out = sl;
   return sl;
 }
 
-// Sink slots of (b, h), by one warp after build_block_layout: s_sinks[i], i < sl.n_sinks,
-// is sink i, or -1 when it is dropped -- out of range, inside the current block [g0, g1),
-// a repeat of the previous entry (the list is ascending among its valid entries) or
-// inside a kept block. bs_div divides by bs (exact below L).
+// Sink slots of (b, h), by one warp after build_block_layout: s_sinks[i], i < sl.n_sinks
+// (slot sink_start + i), is sink i, or -1 when it is dropped -- out of range, inside the
+// current block [g0, g1), a repeat of the previous entry (the list is ascending among its
+// valid entries) or inside a kept block. bs_div divides by bs (exact below L).
 __device__ __forceinline__ void dedupe_sinks(const LayoutPrefetch& pf, const int32_t* snk_g, const SlotLayout& sl,
                                              int L, int P, int g0, int g1, const FastDiv& bs_div, const int* s_blk,
                                              int* s_sinks) {
@@ -148,8 +149,8 @@ __device__ __forceinline__ void dedupe_sinks(const LayoutPrefetch& pf, const int
 template <bool SPARSE>
 __device__ __forceinline__ int group_key0(const SlotLayout& sl, const int* s_blk, int bs, int g0, int gs) {
   if (!SPARSE) return gs;
-  if (gs < sl.gen_start || gs >= sl.n_slots) return -1;
-  if (gs < sl.blk_start) return g0 + (gs - sl.gen_start);
+  if (gs >= sl.sink_start) return -1;
+  if (gs < sl.blk_start) return g0 + gs;
   const int rel = gs - sl.blk_start;
   const int i = static_cast<int>(sl.pad_div.div(static_cast<uint32_t>(rel)));
   return s_blk[i] * bs + (rel - i * sl.pad_bs);
@@ -157,16 +158,19 @@ __device__ __forceinline__ int group_key0(const SlotLayout& sl, const int* s_blk
 
 // Key of a sink-segment slot, or -1 for padding and dropped sinks.
 __device__ __forceinline__ int sink_slot_key(const SlotLayout& sl, const int* s_sinks, int slot) {
-  return (slot >= 0 && slot < sl.n_sinks) ? s_sinks[slot] : -1;
+  const int i = slot - sl.sink_start;
+  return (i >= 0 && i < sl.n_sinks) ? s_sinks[i] : -1;
 }
 
 // Whether a slot holds a key of the set (not padding, not a dropped sink, not past the end).
 template <bool SPARSE>
 __device__ __forceinline__ bool slot_valid(const SlotLayout& sl, const int* s_sinks, int L, int bs, int G, int slot) {
   if (!SPARSE) return slot < L;
-  if (slot < sl.gen_start) return slot < sl.n_sinks && s_sinks[slot] >= 0;
-  if (slot < sl.blk_start) return (slot - sl.gen_start) < G;
-  if (slot >= sl.n_slots) return false;
+  if (slot < sl.blk_start) return slot < G;
+  if (slot >= sl.sink_start) {
+    const int i = slot - sl.sink_start;
+    return i < sl.n_sinks && s_sinks[i] >= 0;
+  }
   const int rel = slot - sl.blk_start;
   const int i = static_cast<int>(sl.pad_div.div(static_cast<uint32_t>(rel)));
   const int r = rel - i * sl.pad_bs;

@@ -164,11 +164,13 @@ FOCUS_API size_t focus_dense_workspace_bytes(int B, int Hq, int Hkv, int L, int 
  * active queries (as focus_dense_attention), the sink importance colsum [B, Hkv, L] (as its
  * colsum_opt) and the sinks [B, Hkv, S] = top-min(S, L) columns of colsum per KV head,
  * ascending, -1 tail (as focus_sink_identify). Where the few-query kernel serves the shape
- * (d = 128, (Hq/Hkv) * qcap <= 64) the three run in one launch: after the cluster merge the
- * kernel re-reads its K tiles, most recent first, for the column sums and selects the sinks
- * within the cluster; other shapes run the calls in sequence (colsum and sinks are then
- * still both written). colsum and sinks are required. Requires 1 <= S <= 4096 and the
- * conditions of focus_dense_attention with column sums; ws/ws_bytes as there.
+ * (d = 128, (Hq/Hkv) * qcap <= 64) the attention and the column sums run in one launch:
+ * after the cluster merge the kernel re-reads the K tiles, most recently read first, for
+ * the column sums. The same launch also selects the sinks within the cluster when each of
+ * its CTAs holds at most 2560 columns (L up to about 10K with 4 CTAs per KV head, 20K with
+ * 8) and S <= 512; otherwise the top-S runs as a second launch. Other shapes run the calls
+ * in sequence. colsum and sinks are both written in every case. Requires 1 <= S <= 4096
+ * and the conditions of focus_dense_attention with column sums; ws/ws_bytes as there.
  */
 FOCUS_API int focus_dense_attention_sinks(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K,
                                           const focus_bf16* V, int B, int Hq, int Hkv, int L, int d, int qcap,

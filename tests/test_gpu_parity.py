@@ -318,6 +318,43 @@ def test_sink_layer_cluster_top_s_matches_the_top_s_kernel(F):
     assert assert_index_sets(s2, c1.double().cpu().numpy(), S, "top-S kernel vs one-call column sums") == 0
 
 
+MANY_ROW_CASES = [
+    # B, Hq, Hkv, L, qcap, n_q (None = all rows): enough 256-row blocks for the many-row kernel
+    (1, 16, 16, 2400, 2400, None),          # ragged key tile and ragged row block
+    (2, 8, 4, 2700, 2700, None),            # GQA 2:1, two sequences
+    (2, 16, 16, 3000, 2048, [2048, 1000]),  # valid-row counts: rows past n_q written as zero
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,qcap,n_q", MANY_ROW_CASES)
+def test_dense_attention_many_rows(F, B, Hq, Hkv, L, qcap, n_q):
+    """The many-row dense kernel (P kept in tensor memory, two query tiles per CTA) against
+    the oracle on sampled rows of every head."""
+    d = 128
+    Q = inputs.random_bf16((B, Hq, qcap, d), seed=7 * L + qcap, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=7 * L + 1, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=7 * L + 2, device=DEV)
+    O = torch.full((B, Hq, qcap, d), 5.0, dtype=torch.bfloat16, device=DEV)
+    nq = None if n_q is None else torch.tensor(n_q, dtype=torch.int32, device=DEV)
+    F.focus_dense_attention(Q, nq, K, V, O)
+    torch.cuda.synchronize()
+    assert F.device_error() == 0
+    rng = np.random.default_rng(L)
+    rows = np.sort(np.unique(np.concatenate([rng.choice(qcap, 40, replace=False), [0, qcap - 1]])))
+    ridx = torch.as_tensor(rows, device=DEV)
+    valid = [qcap] * B if n_q is None else n_q
+    scale = float(np.float32(1 / math.sqrt(d)))
+    g = Hq // Hkv
+    for hq in range(Hq):
+        h = hq // g
+        q = inputs.to_f64(Q[:, hq:hq + 1, ridx])
+        ref, _, _ = orc.dense_attention(q, None, inputs.to_f64(K[:, h:h + 1]), inputs.to_f64(V[:, h:h + 1]), scale)
+        for b in range(B):
+            keep = rows < valid[b]
+            ref[b, :, ~keep] = 0.0                 # rows past the valid count are written as zero
+        assert_attention_close(O[:, hq:hq + 1, ridx], ref, what=f"many-row dense head {hq}")
+
+
 def test_dense_attention_planted_sinks_recovered(F):
     cfg = configs.TINY
     st = inputs.step_state(cfg)
