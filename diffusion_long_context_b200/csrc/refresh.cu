@@ -217,7 +217,8 @@ __global__ void __launch_bounds__(kRfThreads, 1)
         tc_fence_after();
         pv(0, j);
         if (more) {
-          if (!mbar_wait(&bk->k_full[kn], ((j + 1) / kRfKStages) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA)) break;
+          if (!mbar_wait(&bk->k_full[kn], ((j + 1) / kRfKStages) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_MMA))
+            break;
           tc_fence_after();
           qk(0, j + 1);
         }
@@ -251,22 +252,30 @@ __global__ void __launch_bounds__(kRfThreads, 1)
         break;
       }
       tc_fence_after();
-      float sv[128];
+      // the raw scores of this row (the four loads in flight together); the scale is applied
+      // inside the exponent's FFMA, and the maximum is taken on raw scores (scale > 0)
+      uint32_t sr[128];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(sr));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(sr + 64));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(sr + 96));
+      tmem_ld_wait();
+      float* sv = reinterpret_cast<float*>(sr);
+      const int nvalid = a.L - j * 128;             // keys of this tile inside [0, L)
+      if (nvalid < 128) {                           // only the last tile can be partial
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t rg[32];
-        tmem_ld32(tS + c * 32, rg);
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) sv[c * 32 + k] = __uint_as_float(rg[k]) * a.scale_log2;
+        for (int k = 0; k < 128; ++k)
+          if (k >= nvalid) sv[k] = -INFINITY;
       }
-      const int nvalid = min(128, a.L - j * 128);   // keys of this tile inside [0, L)
-      float mt = -INFINITY;
+      // the row maximum over eight independent chains (max is exact in any order)
+      float mx[8];
 #pragma unroll
-      for (int k = 0; k < 128; ++k) {
-        if (k >= nvalid) sv[k] = -INFINITY;
-        mt = fmaxf(mt, sv[k]);
-      }
+      for (int u = 0; u < 8; ++u) mx[u] = sv[u];
+#pragma unroll
+      for (int k = 8; k < 128; ++k) mx[k & 7] = fmaxf(mx[k & 7], sv[k]);
+      const float mr =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float mt = mr * a.scale_log2;
       // keep the reference maximum unless it grows by more than 2^8 (p stays <= 256)
       float alpha = 1.f;
       bool rescale = false;
@@ -275,22 +284,25 @@ __global__ void __launch_bounds__(kRfThreads, 1)
         m_ref = mt;
         rescale = true;
       }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      const float c2 = a.scale_log2;
       // P over the first 64 columns of S_i, 32 keys at a time. This thread has read its whole
       // row of S, and PV_i(j - 1), which read the previous P, completed before QK_i(j)
       // signalled s_full.
-      float ls = 0.f;
+      float lsc[4] = {0.f, 0.f, 0.f, 0.f};           // four independent row-sum chains
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float p0 = exp2_approx(sv[32 * c + 2 * k] - m_use), p1 = exp2_approx(sv[32 * c + 2 * k + 1] - m_use);
-          ls += p0 + p1;
+          const float p0 = exp2_approx(fmaf(sv[32 * c + 2 * k], c2, neg_m));
+          const float p1 = exp2_approx(fmaf(sv[32 * c + 2 * k + 1], c2, neg_m));
+          lsc[k & 3] += p0 + p1;
           pk[k] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);
       }
+      const float ls = (lsc[0] + lsc[1]) + (lsc[2] + lsc[3]);
       l_sum = l_sum * alpha + ls;
       if (j > 0 && __any_sync(0xffffffffu, rescale && alpha != 1.f)) {
         // O_i must hold PV_i(j - 1) before its rows are rescaled
