@@ -45,7 +45,7 @@ bool decode_fused_supported(int d, int Hq, int Hkv, int qcap, int L, int S, int 
 bool refresh_supported(int d, int B, int Hq, int Hkv, int qcap, int sms);
 int refresh_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                       __nv_bfloat16* O, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
-                      cudaStream_t stream);
+                      cudaStream_t stream, float* kbar = nullptr, int P = 0, int bs = 1);
 
 constexpr int kBM = 128;            // query rows per CTA (tcgen05 M)
 constexpr int kBN = 128;            // keys per tile
@@ -1048,6 +1048,30 @@ extern "C" int focus_dense_attention_sinks(const focus_bf16* Q, const int32_t* n
                 : run_attention<64, false>(a, plan, ws, colsum, s, sinks, S, &done);
   if (st != FOCUS_OK || done) return st;
   return focus_sink_identify(colsum, B, Hkv, L, S, sinks, stream);   // the top-S as its own launch
+}
+
+extern "C" int focus_full_refresh(const focus_bf16* Q, const focus_bf16* K, const focus_bf16* V, int B, int Hq,
+                                  int Hkv, int L, int d, float scale, focus_bf16* O, int P, int bs, float* kbar,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  int st = check_common(Q, K, V, O, B, Hq, Hkv, L, d, L);
+  if (st != FOCUS_OK) return st;
+  FOCUS_CHECK_ARG(kbar, "null pointer argument");
+  FOCUS_CHECK_ARG(1 <= P && P <= L && bs >= 1, "need 1 <= P <= L and bs >= 1 (P=%d bs=%d L=%d)", P, bs, L);
+  FOCUS_CHECK_ARG(aligned16(kbar), "kbar must be 16-byte aligned");
+  if (d != 64 && d != 128) {
+    set_error("head dim %d unsupported (64 or 128)", d);
+    return FOCUS_ERR_UNSUPPORTED;
+  }
+  if (B == 0) return FOCUS_OK;
+  if (refresh_supported(d, B, Hq, Hkv, L, device_sm_count()) && 128 % bs == 0)
+    return refresh_attention(reinterpret_cast<const __nv_bfloat16*>(Q), nullptr,
+                             reinterpret_cast<const __nv_bfloat16*>(K), reinterpret_cast<const __nv_bfloat16*>(V),
+                             reinterpret_cast<__nv_bfloat16*>(O), B, Hq, Hkv, L, L, scale * kLog2e,
+                             static_cast<cudaStream_t>(stream), kbar, P, bs);
+  // other shapes: the dense attention and the block means as two launches
+  st = focus_dense_attention(Q, nullptr, K, V, B, Hq, Hkv, L, d, L, scale, O, nullptr, ws, ws_bytes, stream);
+  if (st != FOCUS_OK) return st;
+  return focus_block_means(K, B, Hkv, L, d, P, bs, kbar, stream);
 }
 
 extern "C" size_t focus_sparse_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int acap, int S, int C, int bs,

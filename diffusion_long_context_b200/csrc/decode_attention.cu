@@ -322,8 +322,8 @@ __device__ __noinline__ void decode_sink_topk(const DecArgs& a, DecBook* bk, uin
 
 template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM>
 __global__ void __launch_bounds__(kDecThreads, 1)
-    decode_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ DecArgs a) {
+    decode_attn_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ DecArgs a) {
   using SM = DecSmem<NQ, STAGES>;
   constexpr int D = kDecD;
   constexpr int CH = D / 8;
@@ -496,7 +496,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       bk->abort_flag = 0;
       if (rank == 0) bk->tile_ctr = static_cast<uint32_t>(cs * STAGES);
       fence_mbar_init();
-      if (FUSED) tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
@@ -527,21 +526,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   // query rows (into the idle K ring) and its first round of block means (into the idle V
   // ring) by bulk copies, issued before anything else.
   constexpr int kKbRound = STAGES >= 3 ? 128 : 120;            // kbar rows per round
-  // One slice: the group's rows go by TMA straight into the MMA's SW128 Q operand, and qbar
-  // is summed from there. Several slices: every slice needs all the group's rows for qbar,
-  // so they are bulk-copied raw into the K ring and the slice's rows laid out from there.
-  const bool q_direct = a.n_slices == 1;
+  // (Measured: loading the slice's rows by TMA straight into the SW128 operand and summing
+  // qbar from there took 0.2 us longer than the raw copy and the layout pass below.)
   if (FUSED && threadIdx.x == 0) {
-    if (q_direct) {
-      mbar_arrive_expect_tx(&bk->q_bar, static_cast<uint32_t>(NQ * D * 2));
-      for (int at = 0; at < D / 64; ++at)
-        tma_load_3d(smem_u32(sQ + at * (NQ * 128)), &tmQ, &bk->q_bar, at * 64, 0, bh);
-    } else {
-      const uint32_t qbytes = static_cast<uint32_t>(a.g * a.qcap * D * 2);
-      mbar_arrive_expect_tx(&bk->q_bar, qbytes);
-      bulk_load(smem_u32(sK), a.Q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * a.g) * a.qcap * D,
-                qbytes, &bk->q_bar);
-    }
+    const uint32_t qbytes = static_cast<uint32_t>(a.g * a.qcap * D * 2);
+    mbar_arrive_expect_tx(&bk->q_bar, qbytes);
+    bulk_load(smem_u32(sK), a.Q + (static_cast<size_t>(b) * a.Hq + static_cast<size_t>(kvh) * a.g) * a.qcap * D,
+              qbytes, &bk->q_bar);
     if (j_begin < j_end) {
       const int nrow = min(kKbRound, j_end - j_begin);
       mbar_arrive_expect_tx(&bk->kb_bar, static_cast<uint32_t>(nrow * D * 4));
@@ -588,16 +579,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_wait(&bk->q_bar, 0, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_PRODUCER);
       int i = rg;                                   // rg < RG <= qcap is not assumed
       while (i >= a.qcap) i -= a.qcap;
-      // dims 2dp, 2dp + 1 of row r: in the staged raw rows, or in 16-byte chunk dp / 4 of
-      // row r of the SW128 operand
-      const uint32_t sw_in = static_cast<uint32_t>((dp & 3) * 4);
 #pragma unroll 4
       for (int r = rg; r < nr; r += RG) {
         if (i < nq_b) {
-          const __nv_bfloat162 v =
-              q_direct ? *reinterpret_cast<const __nv_bfloat162*>(sQ + sw128_offset(r, dp >> 2, NQ) + sw_in)
-                       : s_qrows[r * (D / 2) + dp];
-          const float2 f = __bfloat1622float2(v);
+          const float2 f = __bfloat1622float2(s_qrows[r * (D / 2) + dp]);
           acc.x += f.x;
           acc.y += f.y;
         }
@@ -607,10 +592,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       s_part[rg * D + 2 * dp] = acc.x;
       s_part[rg * D + 2 * dp + 1] = acc.y;
     }
-    // several slices: this slice's rows as the MMA's K-major SW128 Q operand, from the
-    // staged copy (the fence after the top-C orders these writes before the tensor cores
-    // read them)
-    for (int idx = threadIdx.x; !q_direct && idx < NQ * CH; idx += kDecThreads) {
+    // this slice's rows as the MMA's K-major SW128 Q operand, from the staged copy (the
+    // fence after the top-C orders these writes before the tensor cores read them)
+    for (int idx = threadIdx.x; idx < NQ * CH; idx += kDecThreads) {
       const int q = idx / CH, c = idx % CH;
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (q < n_rows) {
@@ -1264,17 +1248,11 @@ bool plan_sink_topk(int L, int S, int cs, int* chunk, int* kpt) {
 template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM = false>
 int run_decode(const DecArgs& a0, cudaStream_t stream, bool* sinks_done = nullptr) {
   DecArgs a = a0;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mk, mv;
   int st = dec_make_map(&mk, a.K, a.B * a.Hkv, a.L, a.box_rows);
   if (st != FOCUS_OK) return st;
   st = dec_make_map(&mv, a.V, a.B * a.Hkv, a.L, a.box_rows);
   if (st != FOCUS_OK) return st;
-  mq = mk;                                         // read only by the fused form
-  if (FUSED) {
-    // the group's g * qcap rows, NQ-row boxes (rows past the group read as zeros)
-    st = dec_make_map(&mq, a.Q, a.B * a.Hkv, a.g * a.qcap, NQ);
-    if (st != FOCUS_OK) return st;
-  }
   a.dev_err = device_error_word();
   a.n_slices = (a.g * a.qcap + NQ - 1) / NQ;
   const int units = a.B * a.Hkv * a.n_slices;
@@ -1293,8 +1271,7 @@ int run_decode(const DecArgs& a0, cudaStream_t stream, bool* sinks_done = nullpt
                                                  "decode attention"))
     return st_attr;
   const cudaError_t e =
-      launch_k_cluster(kern, dim3(cs, units), dim3(kDecThreads), DecSmem<NQ, STAGES>::kBytes, stream, cs, mq, mk, mv,
-                       a);
+      launch_k_cluster(kern, dim3(cs, units), dim3(kDecThreads), DecSmem<NQ, STAGES>::kBytes, stream, cs, mk, mv, a);
   note_launch();
   if (e != cudaSuccess) {
     set_error("decode attention launch: %s", cudaGetErrorString(e));

@@ -19,6 +19,18 @@
 // S_i only after PV_i(j) has read P_i). Each row keeps a reference maximum m: p = 2^(s - m)
 // while every s stays below m + 8; a tile that would exceed it moves m up and rescales the
 // row of O_i in tensor memory (after PV_i(j-1) has landed). Row sums are per-thread.
+// The two warpgroups take turns on the exponential unit (16 ex2 per clock per SM: a tile's
+// 2 x 16384 exponentials take about as many clocks as its four MMAs): warpgroup 1 starts the
+// exponentials of tile j once warpgroup 0 has finished its own, and warpgroup 0 those of
+// tile j + 1 once warpgroup 1 has finished tile j, so one warpgroup's exponentials overlap
+// the other's MMAs instead of both groups contending at once and then waiting together.
+//
+// Block entry (method steps (4): a prompt block is represented by the mean of its keys,
+// computed once per generation block): with kbar requested, the K tiles that stream through
+// the CTAs anyway also give the block means. K tile t of the prompt is summed by row block
+// t mod (row blocks of the head) -- every row block of a head streams every tile, so each
+// tile is summed exactly once -- by the producer warp, between issuing tile t + 1 and
+// refilling t's ring stage.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,6 +54,10 @@ struct RfArgs {
   int rows;                // g * qcap rows per KV group
   float scale_log2;
   int* dev_err;
+  // block means of the prompt (block entry): kbar [B, Hkv, nb, 128] fp32 of the blocks
+  // [j*bs, min(P, (j+1)*bs)), bs dividing 128; null when not wanted
+  float* kbar;
+  int P, bs, nb;
 };
 
 struct __align__(8) RfBook {
@@ -49,6 +65,7 @@ struct __align__(8) RfBook {
   uint64_t k_full[kRfKStages], k_empty[kRfKStages];
   uint64_t v_full[kRfVStages], v_empty[kRfVStages];
   uint64_t s_full[2], p_full[2], o_done[2], drain;
+  uint64_t tok[2];         // exponential phase of a tile done by warpgroup 0 / 1
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -119,6 +136,8 @@ __global__ void __launch_bounds__(kRfThreads, 1)
         mbar_init(&bk->o_done[i], 1);
       }
       mbar_init(&bk->drain, 1);
+      mbar_init(&bk->tok[0], 4);
+      mbar_init(&bk->tok[1], 4);
       bk->abort_flag = 0;
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
@@ -138,6 +157,39 @@ __global__ void __launch_bounds__(kRfThreads, 1)
 
   if (warp == kRfProducerWarp) {
     // ------------------------------------------------------------ producer
+    // Lane 0 issues the copies; with kbar requested the whole warp sums this CTA's prompt
+    // tiles (lane l: dims 4l .. 4l+3 of every row, read from the SW128 tile).
+    const int n_ptiles = a.kbar ? (a.P + 127) / 128 : 0;
+    auto block_means_of = [&](int t) {
+      if (t >= n_ptiles || t % static_cast<int>(gridDim.x) != static_cast<int>(blockIdx.x)) return true;
+      const int ks = t % kRfKStages;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bk->k_full[ks], (t / kRfKStages) & 1, abort_flag, a.dev_err,
+                                             DEV_ERR_TIMEOUT_PRODUCER)))
+        return false;
+      const uint8_t* tile = sK + ks * SM::kTile;
+      const int c = lane >> 1;                                // 16-byte chunk of the row
+      const uint32_t base = static_cast<uint32_t>((c >> 3) * (128 * 128) + (lane & 1) * 8);
+      for (int r0 = 0; r0 < 128; r0 += a.bs) {
+        const int blk = (t * 128 + r0) / a.bs;
+        const int n = min(a.bs, a.P - blk * a.bs);            // valid rows of the block
+        if (n <= 0) break;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = r0; r < r0 + n; ++r) {
+          const uint2 v = *reinterpret_cast<const uint2*>(tile + base + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+          const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.x));
+          const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&v.y));
+          acc.x += f0.x;
+          acc.y += f0.y;
+          acc.z += f1.x;
+          acc.w += f1.y;
+        }
+        const float inv = 1.f / static_cast<float>(n);
+        reinterpret_cast<float4*>(a.kbar + (static_cast<size_t>(bh) * a.nb + blk) * D)[lane] =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      }
+      return true;
+    };
+    int k_issued = 0, v_issued = 0;
     if (lane == 0) {
       // no evict-first hint: the other row blocks of the same KV head, resident at the same
       // time, read the same K and V tiles out of L2
@@ -145,24 +197,38 @@ __global__ void __launch_bounds__(kRfThreads, 1)
       for (int t = 0; t < 2; ++t)
         for (int at = 0; at < 2; ++at)
           tma_load_3d(smem_u32(sQ + t * SM::kTile + at * (128 * 128)), &tmQ, &bk->q_full, at * 64, m0 + t * 128, bh);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < n_kt; ++j) {
-        const int ks = j % kRfKStages, vs = j % kRfVStages;
+    }
+    bool ok = true;
+    for (int j = 0; j < n_kt && ok; ++j) {
+      const int ks = j % kRfKStages, vs = j % kRfVStages;
+      if (lane == 0) {
         if (j >= kRfKStages &&
             !mbar_wait(&bk->k_empty[ks], ((j / kRfKStages) - 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_PRODUCER))
-          break;
-        mbar_arrive_expect_tx(&bk->k_full[ks], SM::kTile);
-        for (int at = 0; at < 2; ++at)
-          tma_load_3d(smem_u32(sK + ks * SM::kTile + at * (128 * 128)), &tmK, &bk->k_full[ks], at * 64, j * 128, bh);
-        ++k_issued;
-        if (j >= kRfVStages &&
+          ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&bk->k_full[ks], SM::kTile);
+          for (int at = 0; at < 2; ++at)
+            tma_load_3d(smem_u32(sK + ks * SM::kTile + at * (128 * 128)), &tmK, &bk->k_full[ks], at * 64, j * 128,
+                        bh);
+          ++k_issued;
+        }
+        if (ok && j >= kRfVStages &&
             !mbar_wait(&bk->v_empty[vs], ((j / kRfVStages) - 1) & 1, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_PRODUCER))
-          break;
-        mbar_arrive_expect_tx(&bk->v_full[vs], SM::kTile);
-        for (int at = 0; at < 2; ++at)
-          tma_load_3d(smem_u32(sV + vs * SM::kTile + at * (128 * 128)), &tmV, &bk->v_full[vs], at * 64, j * 128, bh);
-        ++v_issued;
+          ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&bk->v_full[vs], SM::kTile);
+          for (int at = 0; at < 2; ++at)
+            tma_load_3d(smem_u32(sV + vs * SM::kTile + at * (128 * 128)), &tmV, &bk->v_full[vs], at * 64, j * 128,
+                        bh);
+          ++v_issued;
+        }
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // tile j - 1 has been issued a ring's depth before its stage is refilled (by this warp)
+      if (ok && j >= 1) ok = block_means_of(j - 1);
+    }
+    if (ok && n_kt >= 1) block_means_of(n_kt - 1);
+    if (lane == 0) {
       // never leave with copies in flight
       rf_wait_drain(&bk->q_full, 0);
       for (int j = max(0, k_issued - kRfKStages); j < k_issued; ++j)
@@ -286,6 +352,15 @@ __global__ void __launch_bounds__(kRfThreads, 1)
       }
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const float c2 = a.scale_log2;
+      // take turns on the exponential unit with the other warpgroup
+      if (wg == 1 || j > 0) {
+        const uint32_t par = static_cast<uint32_t>(wg == 1 ? j : j - 1) & 1u;
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&bk->tok[wg ^ 1], par, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_SOFTMAX))) {
+          ok = false;
+          break;
+        }
+      }
       // P over the first 64 columns of S_i, 32 keys at a time. This thread has read its whole
       // row of S, and PV_i(j - 1), which read the previous P, completed before QK_i(j)
       // signalled s_full.
@@ -303,6 +378,8 @@ __global__ void __launch_bounds__(kRfThreads, 1)
         tmem_st16(tS + c * 16, pk);
       }
       const float ls = (lsc[0] + lsc[1]) + (lsc[2] + lsc[3]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bk->tok[wg]);     // this tile's exponentials are done
       l_sum = l_sum * alpha + ls;
       if (j > 0 && __any_sync(0xffffffffu, rescale && alpha != 1.f)) {
         // O_i must hold PV_i(j - 1) before its rows are rescaled
@@ -419,7 +496,7 @@ bool refresh_supported(int d, int B, int Hq, int Hkv, int qcap, int sms) {
 
 int refresh_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfloat16* K, const __nv_bfloat16* V,
                       __nv_bfloat16* O, int B, int Hq, int Hkv, int L, int qcap, float scale_log2,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, float* kbar, int P, int bs) {
   RfArgs a{};
   a.n_q = n_q;
   a.O = O;
@@ -432,6 +509,10 @@ int refresh_attention(const __nv_bfloat16* Q, const int32_t* n_q, const __nv_bfl
   a.rows = a.g * qcap;
   a.scale_log2 = scale_log2;
   a.dev_err = device_error_word();
+  a.kbar = kbar;
+  a.P = P;
+  a.bs = bs;
+  a.nb = kbar ? (P + bs - 1) / bs : 0;
   CUtensorMap mq, mk, mv;
   int st = rf_make_map(&mq, Q, B * Hkv, a.rows);
   if (st != FOCUS_OK) return st;

@@ -43,6 +43,7 @@ _SIGS = {
     "focus_dense_attention": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "focus_dense_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "focus_dense_attention_sinks": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _i, _p, _p, _sz, _p]),
+    "focus_full_refresh": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _f, _p, _i, _i, _p, _p, _sz, _p]),
     "focus_sink_identify": (_i, [_p, _i, _i, _i, _i, _p, _p]),
     "focus_sparse_attention": (_i, [_p, _p, _p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _i, _f,
                                     _p, _p, _sz, _p]),
@@ -229,6 +230,24 @@ def focus_dense_attention_sinks(Q, n_q, K, V, O, colsum, sinks, scale=None, ws=N
                                          _ptr(O), _ptr(colsum), sinks.shape[2], _ptr(sinks), _ptr(ws), ws_bytes,
                                          _stream(stream))
     _check(st, "focus_dense_attention_sinks")
+
+
+def focus_full_refresh(Q, K, V, O, P, bs, kbar, scale=None, ws=None, stream=None):
+    """Block entry: dense attention of every query (O [B, Hq, L, d]) and the prompt's block
+    means kbar [B, Hkv, ceil(P / bs), d] fp32, in one launch where the kernel serves it."""
+    _need(Q, torch.bfloat16, "Q", 4)
+    _need(K, torch.bfloat16, "K", 4)
+    _need(V, torch.bfloat16, "V", 4)
+    _need(O, torch.bfloat16, "O", 4)
+    _need(kbar, torch.float32, "kbar", 4)
+    B, Hq, L, d = Q.shape
+    Hkv = K.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = dense_workspace_bytes(B, Hq, Hkv, L, d, L, False)
+    ws, ws_bytes = _workspace(need, Q.device, ws)
+    st = lib.focus_full_refresh(_ptr(Q), _ptr(K), _ptr(V), B, Hq, Hkv, L, d, float(scale), _ptr(O), P, bs, _ptr(kbar),
+                                _ptr(ws), ws_bytes, _stream(stream))
+    _check(st, "focus_full_refresh")
 
 
 def focus_sink_identify(colsum, S, sinks, stream=None):

@@ -78,15 +78,28 @@ class SparseStep:
         self.mask.copy_(mask, non_blocking=non_blocking)
 
     # ------------------------------------------------------------------ block entry
-    def block_entry(self):
-        """Block means of every sparse layer (cached for the later steps of the block)."""
+    def block_entry(self, O_full: Optional[torch.Tensor] = None):
+        """Block entry. Without O_full: the block means of every sparse layer only (cached for
+        the later steps of the block). With O_full [B, Hq, L, d]: the block-entry step proper,
+        every layer's dense full refresh into O_full (reused per layer), the sparse layers'
+        block means computed in the same launch."""
         c = self.cfg
-        for l in self.sparse_layers:
-            F.focus_block_means(self.K[l], c.P, c.bs, self.kbar[l])
+        if O_full is None:
+            for l in self.sparse_layers:
+                F.focus_block_means(self.K[l], c.P, c.bs, self.kbar[l])
+            return
+        for l in range(c.n_layers):
+            self.full_refresh_layer(l, O_full)
 
     def full_refresh_layer(self, l: int, O_full: torch.Tensor):
-        """Dense full refresh of layer l: every query of the sequence over all L keys."""
-        F.focus_dense_attention(self.Q_full[l], None, self.K[l], self.V[l], O_full, scale=self.scale)
+        """Dense full refresh of layer l: every query of the sequence over all L keys (with the
+        layer's block means when it is a sparse layer)."""
+        c = self.cfg
+        if l in self.kbar:
+            F.focus_full_refresh(self.Q_full[l], self.K[l], self.V[l], O_full, c.P, c.bs, self.kbar[l],
+                                 scale=self.scale)
+        else:
+            F.focus_dense_attention(self.Q_full[l], None, self.K[l], self.V[l], O_full, scale=self.scale)
 
     # ------------------------------------------------------------------ sparse step
     def select(self):

@@ -160,6 +160,23 @@ FOCUS_API int focus_dense_attention(const focus_bf16* Q, const int32_t* n_q, con
 FOCUS_API size_t focus_dense_workspace_bytes(int B, int Hq, int Hkv, int L, int d, int qcap, int want_colsum);
 
 /*
+ * Block entry in one call -- "半自回归重遮蔽策略" (semi-AR remasking: at block entry the whole
+ * sequence runs dense attention) and method steps (4) (a prompt block is represented by the
+ * mean of its keys, computed once per generation block): O = dense attention of all L
+ * queries of Q [B, Hq, L, d] over all L keys (as focus_dense_attention with n_q = NULL,
+ * qcap = L) and kbar [B, Hkv, nb, d] fp32 = the block means of the prompt [0, P) in blocks of
+ * bs (as focus_block_means). Where the many-row kernel serves the shape (d = 128, enough
+ * 256-row blocks to fill the GPU) and bs divides 128, the block means are summed from the K
+ * tiles the attention streams anyway: one launch, no second read of K. Otherwise the two
+ * calls run in sequence; ws/ws_bytes then serve the dense attention (size them with
+ * focus_dense_workspace_bytes(B, Hq, Hkv, L, d, L, 0)). Requires 1 <= P <= L, bs >= 1,
+ * kbar 16-byte aligned and the conditions of focus_dense_attention.
+ */
+FOCUS_API int focus_full_refresh(const focus_bf16* Q, const focus_bf16* K, const focus_bf16* V, int B, int Hq,
+                                 int Hkv, int L, int d, float scale, focus_bf16* O, int P, int bs, float* kbar,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
  * (3) The sink layer in one call -- method steps (3) and core method: dense attention of the
  * active queries (as focus_dense_attention), the sink importance colsum [B, Hkv, L] (as its
  * colsum_opt) and the sinks [B, Hkv, S] = top-min(S, L) columns of colsum per KV head,

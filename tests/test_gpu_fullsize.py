@@ -184,13 +184,19 @@ def test_full_32k_step_as_the_bench_replays_it(F):
 
 
 def test_full_refresh_32k_sampled_rows(F):
-    """Block-entry dense refresh at 32K: all 32768 queries; 96 sampled rows vs the oracle."""
+    """Block entry at 32K (focus_full_refresh, the step's path): all 32768 queries, 96 sampled
+    rows vs the oracle, and the layer's block means vs the oracle."""
     cfg = configs.FULL_32K
     st = inputs.step_state(cfg)
-    Qf, K, V = inputs.make_layer(cfg, 0, DEV, st.sink_pos)
+    Qf, K, V = inputs.make_layer(cfg, 3, DEV, st.sink_pos)
     O = torch.empty((cfg.B, cfg.Hq, cfg.L, cfg.d), dtype=torch.bfloat16, device=DEV)
-    F.focus_dense_attention(Qf, None, K, V, O)
+    kbar = torch.empty((cfg.B, cfg.Hkv, cfg.nb, cfg.d), dtype=torch.float32, device=DEV)
+    F.focus_full_refresh(Qf, K, V, O, cfg.P, cfg.bs, kbar)
     torch.cuda.synchronize()
+    assert F.device_error() == 0
+    ref_kbar = orc.block_means(inputs.to_f64(K), cfg.P, cfg.bs)
+    got = kbar.cpu().double().numpy()
+    assert np.all(np.abs(got - ref_kbar) <= 1e-3 * np.abs(ref_kbar) + 1e-6), "block means off"
     rng = np.random.default_rng(77)
     heads = rng.choice(cfg.Hq, size=3, replace=False)
     rows = np.sort(rng.choice(cfg.L, size=32, replace=False))

@@ -355,6 +355,45 @@ def test_dense_attention_many_rows(F, B, Hq, Hkv, L, qcap, n_q):
         assert_attention_close(O[:, hq:hq + 1, ridx], ref, what=f"many-row dense head {hq}")
 
 
+FULL_REFRESH_CASES = [
+    # B, Hq, Hkv, L, d, P, bs: block entry (attention of every query + block means)
+    (1, 16, 16, 2400, 128, 2336, 64),     # one launch: the means summed from the K stream
+    (2, 8, 4, 2700, 128, 2605, 32),       # GQA, a short last block (2605 = 81 * 32 + 13)
+    (1, 16, 16, 2400, 128, 2300, 128),    # bs = 128: one block per key tile
+    (1, 16, 16, 2400, 128, 2304, 96),     # bs not dividing 128: attention and block means as two calls
+    (1, 4, 4, 600, 64, 500, 64),          # d = 64: two calls
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,d,P,bs", FULL_REFRESH_CASES)
+def test_full_refresh_with_block_means(F, B, Hq, Hkv, L, d, P, bs):
+    """focus_full_refresh: every query over all keys (sampled rows of every head) and the
+    prompt's block means, against the oracle."""
+    Q = inputs.random_bf16((B, Hq, L, d), seed=11 * L + bs, device=DEV)
+    K = inputs.random_bf16((B, Hkv, L, d), seed=11 * L + bs + 1, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=11 * L + bs + 2, device=DEV)
+    nb = -(-P // bs)
+    O = torch.full((B, Hq, L, d), 5.0, dtype=torch.bfloat16, device=DEV)
+    kbar = torch.full((B, Hkv, nb, d), -9.0, dtype=torch.float32, device=DEV)
+    F.focus_full_refresh(Q, K, V, O, P, bs, kbar)
+    torch.cuda.synchronize()
+    assert F.device_error() == 0
+    K64 = inputs.to_f64(K)
+    ref_kbar = orc.block_means(K64, P, bs)
+    got = kbar.cpu().double().numpy()
+    assert np.all(np.abs(got - ref_kbar) <= KBAR_REL * np.abs(ref_kbar) + 1e-6), "block means off"
+    rng = np.random.default_rng(L + bs)
+    rows = np.sort(np.unique(np.concatenate([rng.choice(L, 24, replace=False), [0, L - 1]])))
+    ridx = torch.as_tensor(rows, device=DEV)
+    scale = float(np.float32(1 / math.sqrt(d)))
+    g = Hq // Hkv
+    for hq in range(Hq):
+        h = hq // g
+        q = inputs.to_f64(Q[:, hq:hq + 1, ridx])
+        ref, _, _ = orc.dense_attention(q, None, K64[:, h:h + 1], inputs.to_f64(V[:, h:h + 1]), scale)
+        assert_attention_close(O[:, hq:hq + 1, ridx], ref, what=f"full refresh head {hq}")
+
+
 def test_dense_attention_planted_sinks_recovered(F):
     cfg = configs.TINY
     st = inputs.step_state(cfg)
