@@ -40,7 +40,7 @@ from diffusion_long_context_b200 import configs, inputs  # noqa: E402
 # dominant kernel on the 32K workload, from the committed ncu summaries: the fused sparse
 # layer (default step) and the unfused sparse attention. Each is reset to None whenever
 # its kernel changes, until it is captured again; other workloads report None.
-TRAFFIC_BYTES = {"fused": 78.27e6, "sparse": None}
+TRAFFIC_BYTES = {"fused": 78.27e6, "sparse": 69.61e6}
 METRIC = "sparse dLLM attn step latency & active tok/s at 32K ctx; % of HBM/TC roofline"
 WORKLOADS = {"full32k": configs.FULL_32K, "llada8k": configs.LLADA_8K, "dream16k": configs.DREAM_16K}
 L2_BYTES = 126 * 1024 * 1024

@@ -80,8 +80,6 @@ struct DecArgs {
   float* colsum;
   int32_t* sinks_out;
   int S_out;
-  int ts_chunk;                // columns per CTA for the top-S (a multiple of 4)
-  int ts_kpt;                  // columns per thread for it (8)
 };
 
 struct __align__(8) DecBook {
@@ -152,16 +150,19 @@ __device__ __noinline__ void dec_top_c_large(const uint32_t* s_key, int nb, int 
 //   colsum[b, h, key] = sum over query columns q of 2^(scale_log2 * s[key, q] - lse2[q]).
 // CTA r takes the 128-key tiles p_n - 1 - r, p_n - 1 - r - cs, ...: from the last tile
 // down (the tiles the attention pass read last first), with no claim round trip on the
-// producer's path. The pass re-reads K from HBM: an evict-last hint on the attention
-// pass's K loads (V evict-first) was measured to leave the column-sum pass at the same
-// 6.1 TB/s, i.e. no reuse out of L2 at this size (268 MB of K at 32K). K tiles flow through a CS-slot ring
+// producer's path. The pass re-reads K from HBM: an evict-last or evict-normal hint on the
+// attention pass's K loads (V evict-first) was measured to leave the column-sum pass at the
+// same 6.1 TB/s or slower, i.e. no reuse out of L2 at this size (268 MB of K at 32K).
+// K tiles flow through a CS-slot ring
 // made of the K ring and the V-ring stages the merge does not read; S^T = K_tile . Q^T
 // lands in the two S buffers of tensor memory; each softmax thread owns one key, the two
 // query halves of a key are added through shared memory, and the key's sum is stored.
+// Each key lane also keeps the largest sum it produced (one per tile residue it % m,
+// m = ceil(S / 128)) in gmax: the bound decode_sink_topk starts from.
 template <int NQ, int STAGES>
 __device__ __noinline__ void decode_colsum_phase(const CUtensorMap* tmK, const DecArgs& a, DecBook* bk, uint8_t* sK,
                                                  uint8_t* sV, const uint8_t* sQ, uint32_t tmem, int bh, int rank,
-                                                 int cs) {
+                                                 int cs, uint32_t* gmax) {
   using SM = DecSmem<NQ, STAGES>;
   constexpr int D = kDecD;
   constexpr int QH = NQ / 2;
@@ -238,6 +239,10 @@ __device__ __noinline__ void decode_colsum_phase(const CUtensorMap* tmK, const D
     const int t = threadIdx.x & 127, q0 = (warp >> 2) * QH;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float* hbuf = &bk->red[0][0];              // [2][128]: the second query half's sums
+    // group maxima for the top-S (decode_sink_topk): key lane t, tile residue it % m
+    const int m = max(1, min(4, (a.S_out + 127) / 128));
+    uint32_t gm[4] = {0u, 0u, 0u, 0u};
+    int u = 0;                                 // it % m
     float lse[QH];
 #pragma unroll
     for (int q = 0; q < QH; ++q) lse[q] = bk->lse2[q0 + q];
@@ -260,64 +265,169 @@ __device__ __noinline__ void decode_colsum_phase(const CUtensorMap* tmK, const D
       if (warp >= 4) hbuf[sb * 128 + t] = acc;
       named_bar_sync(1, kDecSoftmaxThreads);
       const int key = tile * 128 + t;
-      if (warp < 4 && key < a.L) a.colsum[static_cast<size_t>(bh) * a.L + key] = acc + hbuf[sb * 128 + t];
+      if (warp < 4 && key < a.L) {
+        const float v = acc + hbuf[sb * 128 + t];
+        a.colsum[static_cast<size_t>(bh) * a.L + key] = v;
+        const uint32_t kv = float_order_key(v);
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+          if (x == u) gm[x] = max(gm[x], kv);
+      }
+      if (++u == m) u = 0;
+    }
+    if (warp < 4)
+      for (int x = 0; x < m; ++x) gmax[x * 128 + t] = gm[x];
+  }
+}
+
+// Top-S sinks of the sink layer's column sums, selected inside the cluster (core method:
+// the sinks found at the sink layer are reused by every deeper layer). Order: larger
+// column sum first, ties to the lower column; the output lists the S columns ascending.
+//
+// Each CTA selects the top-S of the columns its own column-sum pass produced (its tiles
+// t0, t0 + cs, ...), then CTA 0 selects the top-S of the cs * S candidates:
+//  1. A lower bound T of this CTA's S-th largest column sum: during the pass every key
+//     lane t (and, for S > 128, every tile residue it % m) keeps the maximum of the sums it
+//     produced, so there are 128 * m >= S group maxima, each one of the sums; the S-th
+//     largest of them is at most the S-th largest sum. Every sum of the top-S is >= T.
+//  2. The sums >= T are appended to a candidate list (a shared counter; typically a few
+//     dozen of the 8192 columns at 32K). Each is packed as (order key << 32) | ~column, so
+//     that one 64-bit comparison orders by sum and then by lower column, and all packed
+//     values are distinct.
+//  3. The top-S of the candidates by rank counting (rank = number of larger packed values).
+//     When more candidates than kSinkCand qualify (many equal sums), the CTA runs the
+//     general radix selection over all its columns instead.
+//  4. Each CTA writes its S best into CTA 0 (distributed shared memory); after a cluster
+//     barrier CTA 0 ranks the cs * S candidates the same way and writes the S columns of
+//     the top-S in ascending order.
+constexpr int kSinkCand = 1024;              // candidates a CTA ranks directly
+constexpr int kSinkCand0 = 2048;             // cs * S candidates of the cluster (CTA 0)
+
+__device__ __forceinline__ uint64_t sink_pack(uint32_t key, int col) {
+  return (static_cast<uint64_t>(key) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(col));
+}
+__device__ __forceinline__ int sink_col(uint64_t p) { return static_cast<int>(~static_cast<uint32_t>(p)); }
+
+// Rank of every packed value v[i], i < n, among v[0 .. n) (the number of larger values;
+// the nonzero values are distinct): v[i] goes to out[rank] when rank < k, so out comes out
+// in descending order.
+__device__ __forceinline__ void sink_rank_select(const uint64_t* v, int n, int k, uint64_t* out) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const uint64_t x = v[i];
+    int r = 0;
+    for (int j = 0; j < n; ++j) r += v[j] > x ? 1 : 0;
+    if (r < k) out[r] = x;
+  }
+}
+
+__device__ __noinline__ void decode_sink_topk(const DecArgs& a, DecBook* bk, uint8_t* ws, const uint32_t* gmax, int bh,
+                                              int rank, int cs) {
+  const int S = a.S_out;
+  const int ng = 128 * max(1, min(4, (S + 127) / 128));   // group maxima (decode_colsum_phase)
+  const int p_n = (a.L + 127) / 128;
+  const int last = p_n - 1 - rank;                     // this CTA's highest tile
+  const int n_own = last >= 0 ? last / cs + 1 : 0;
+  const int t0 = last - (n_own - 1) * cs;              // its lowest tile
+  const int n_pos = n_own * 128;                       // its positions, in ascending column order
+  uint64_t* cand = reinterpret_cast<uint64_t*>(ws);                    // [kSinkCand]
+  uint64_t* best = cand + kSinkCand;                                   // [kDecMaxSinks]
+  uint64_t* cand0 = best + kDecMaxSinks;                               // [kSinkCand0] (CTA 0)
+  int* s_cnt = reinterpret_cast<int*>(cand0 + kSinkCand0);
+  uint32_t* s_T = reinterpret_cast<uint32_t*>(s_cnt + 1);
+  int32_t* s_pos = reinterpret_cast<int32_t*>(s_T + 1);                // [kDecMaxSinks] (fallback)
+  const float* row = a.colsum + static_cast<size_t>(bh) * a.L;
+  auto col_of = [&](int pos) { return (t0 + (pos >> 7) * cs) * 128 + (pos & 127); };
+  if (threadIdx.x == 0) {
+    *s_cnt = 0;
+    *s_T = 0u;
+  }
+  for (int i = threadIdx.x; i < S; i += blockDim.x) best[i] = 0ull;
+  __syncthreads();
+  // 1. T = the S-th largest group maximum (equal maxima ranked by group index)
+  for (int i = threadIdx.x; i < ng; i += blockDim.x) {
+    const uint32_t x = gmax[i];
+    int r = 0;
+    for (int j = 0; j < ng; ++j) {
+      const uint32_t y = gmax[j];
+      r += (y > x || (y == x && j < i)) ? 1 : 0;
+    }
+    if (r == S - 1) *s_T = x;
+  }
+  __syncthreads();
+  const uint32_t T = *s_T;
+  // 2. the candidates: this CTA's column sums >= T
+  for (int pos = threadIdx.x; pos < n_pos; pos += blockDim.x) {
+    const int col = col_of(pos);
+    if (col >= a.L) continue;
+    const uint32_t key = float_order_key(__ldcg(row + col));
+    if (key >= T) {
+      const int slot = atomicAdd(s_cnt, 1);
+      if (slot < kSinkCand) cand[slot] = sink_pack(key, col);
     }
   }
-}
-
-// Top-S sinks of the sink layer's column sums, selected by the cluster (core method: the
-// sinks found at the sink layer are reused by every deeper layer). CTA r takes the
-// contiguous columns [r * chunk, r * chunk + chunk) of its (b, h), selects their top-S and
-// pushes the S candidates (order key, column) into CTA 0 in rank order, so the candidate
-// list is in ascending column order and a tie between candidates still resolves to the
-// lower column; CTA 0 selects the top-S of the cs * S candidates. `ws` is the idle K and V
-// rings. The column sums were written by the cluster's CTAs before a fence and a cluster
-// barrier; they are read from L2.
-template <int KPT>
-__device__ __forceinline__ void decode_topk_share(const float* row, int n, int S, uint32_t* s_key, int32_t* s_loc,
-                                                  TopkShared& tk, int* s_priv, int* s_wide) {
-  const int i0 = threadIdx.x * KPT;
-  uint32_t key[KPT];
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) key[j] = (i0 + j < n) ? float_order_key(__ldcg(row + i0 + j)) : 0u;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j)
-    if (i0 + j < n) s_key[i0 + j] = key[j];
-  block_topk_small_regs<KPT>(key, n, S, s_loc, S, tk, s_priv, s_wide);
-}
-
-__device__ __noinline__ void decode_sink_topk(const DecArgs& a, DecBook* bk, uint8_t* ws, int bh, int rank, int cs) {
-  const int chunk = a.ts_chunk, S = a.S_out;
-  const int c0 = rank * chunk;
-  const int n = min(chunk, a.L - c0);          // >= S (host-checked)
-  uint32_t* s_key = reinterpret_cast<uint32_t*>(ws);                          // [chunk]
-  int32_t* s_loc = reinterpret_cast<int32_t*>(s_key + chunk);                 // [S]
-  uint32_t* s_ckey = reinterpret_cast<uint32_t*>(s_loc + S);                  // [cs * S] (CTA 0)
-  int32_t* s_cidx = reinterpret_cast<int32_t*>(s_ckey + static_cast<size_t>(cs) * S);
-  int32_t* s_pos = s_cidx + static_cast<size_t>(cs) * S;                      // [S]
-  int* s_priv = reinterpret_cast<int*>(s_pos + S);                            // per-warp histograms
-  int* s_wide = s_priv + 2 * (kDecThreads / 32) * 257;                        // [2048 + 64]
-  const float* row = a.colsum + static_cast<size_t>(bh) * a.L + c0;
-  decode_topk_share<8>(row, n, S, s_key, s_loc, bk->tk, s_priv, s_wide);   // n <= 8 * threads
   __syncthreads();
-  const uint32_t ck0 = smem_u32(s_ckey), ci0 = smem_u32(s_cidx);
-  for (int i = threadIdx.x; i < S; i += kDecThreads) {
-    const int c = s_loc[i];
-    const uint32_t slot = static_cast<uint32_t>(rank * S + i) * 4u;
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dsmem_addr(ck0 + slot, 0)), "r"(s_key[c]) : "memory");
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dsmem_addr(ci0 + slot, 0)), "r"(c0 + c) : "memory");
+  const int n_cand = *s_cnt;
+  // 3. this CTA's top-S, descending
+  if (n_cand <= kSinkCand) {
+    sink_rank_select(cand, n_cand, S, best);
+  } else {
+    // many equal sums: the radix selection over all of this CTA's columns (ties to the
+    // lower position, i.e. the lower column)
+    auto key_of = [&](int pos) {
+      const int col = col_of(pos);
+      return col < a.L ? float_order_key(__ldcg(row + col)) : 0u;
+    };
+    block_topk_ascending(key_of, n_pos, S, s_pos, S, bk->tk);
+    __syncthreads();
+    for (int i = threadIdx.x; i < S; i += blockDim.x) {
+      const int pos = s_pos[i];
+      const int col = pos >= 0 ? col_of(pos) : a.L;
+      cand[i] = col < a.L ? sink_pack(float_order_key(__ldcg(row + col)), col) : 0ull;
+    }
+    __syncthreads();
+    sink_rank_select(cand, S, S, best);
   }
-  if (cs > 1) cluster_sync();                  // every candidate is in CTA 0
+  __syncthreads();
+  // 4. the S best of every CTA into CTA 0 (list r at cand0[r * S]), then the cluster's top-S
+  const uint32_t c0 = smem_u32(cand0);
+  for (int i = threadIdx.x; i < S; i += blockDim.x)
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(dsmem_addr(c0 + static_cast<uint32_t>(rank * S + i) * 8u, 0)),
+                 "l"(best[i])
+                 : "memory");
+  if (cs > 1) cluster_sync();
   else __syncthreads();
   if (rank != 0) return;
-  const int nc = cs * S;
-  auto ckey = [&](int i) { return s_ckey[i]; };
-  if (nc <= kDecThreads) block_topk_small<1>(ckey, nc, S, s_pos, S, bk->tk, s_wide);
-  else if (nc <= 2 * kDecThreads) block_topk_small<2>(ckey, nc, S, s_pos, S, bk->tk, s_wide);
-  else block_topk_small<4>(ckey, nc, S, s_pos, S, bk->tk, s_wide);
+  // rank of a candidate = its index in its own (descending) list + the entries larger than
+  // it in every other list (binary search); the S of rank < S are the top-S
+  for (int i = threadIdx.x; i < S; i += blockDim.x) best[i] = 0ull;
   __syncthreads();
+  for (int e = threadIdx.x; e < cs * S; e += blockDim.x) {
+    const uint64_t x = cand0[e];
+    if (x == 0ull) continue;
+    const int r = e / S;
+    int rk = e - r * S;
+    for (int o = 0; o < cs; ++o) {
+      if (o == r) continue;
+      const uint64_t* lst = cand0 + o * S;
+      int lo = 0, hi = S;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (lst[mid] > x) lo = mid + 1;
+        else hi = mid;
+      }
+      rk += lo;
+    }
+    if (rk < S) best[rk] = x;
+  }
+  __syncthreads();
+  // the S columns in ascending order (S <= L, so all S are columns)
   int32_t* out = a.sinks_out + static_cast<size_t>(bh) * S;
-  for (int i = threadIdx.x; i < S; i += kDecThreads) out[i] = s_cidx[s_pos[i]];
+  for (int i = threadIdx.x; i < S; i += blockDim.x) {
+    const int ci = sink_col(best[i]);
+    int r = 0;
+    for (int j = 0; j < S; ++j) r += sink_col(best[j]) < ci ? 1 : 0;
+    out[r] = ci;
+  }
 }
 
 template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM>
@@ -1130,7 +1240,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
   }
   if (cs > 1) cluster_arrive_relaxed();   // this warp's reads of the partials are done
-  if constexpr (COLSUM) decode_colsum_phase<NQ, STAGES>(&tmK, a, bk, sK, sV, sQ, tmem, bh, rank, cs);
+  if constexpr (COLSUM)
+    decode_colsum_phase<NQ, STAGES>(&tmK, a, bk, sK, sV, sQ, tmem, bh, rank, cs, reinterpret_cast<uint32_t*>(sP));
   if (cs > 1) cluster_wait();             // no CTA leaves while its partials may still be read
   if constexpr (COLSUM) {
     // the column sums are visible to the whole cluster
@@ -1144,7 +1255,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     }
     // every CTA of the cluster takes the same barriers here, also after a wait ran out (the
     // sinks are then undefined, and the device error word says so)
-    if (a.sinks_out) decode_sink_topk(a, bk, sK, bh, rank, cs);
+    if (a.sinks_out) decode_sink_topk(a, bk, sK, reinterpret_cast<const uint32_t*>(sP), bh, rank, cs);
   }
 }
 
@@ -1230,19 +1341,10 @@ int choose_cluster(int units) {
   return 1;
 }
 
-// Whether the cluster's fused top-S serves S sinks over L columns with cs CTAs; sets the
-// per-CTA share (a multiple of 4 columns) and the columns per thread. The selection's
-// passes cost in proportion to the columns per thread: up to 8 per thread (a 2560-column
-// share) it beats a separate launch (measured at 8K: the sink layer 59 -> 53 us); at
-// 32K's 8192-column shares it took 29 us against about 12 us for the top-S kernel, whose
-// 8-CTA clusters of 512 threads hold 8 columns per thread, so longer rows use that kernel.
-bool plan_sink_topk(int L, int S, int cs, int* chunk, int* kpt) {
-  const int c = ((L + cs - 1) / cs + 3) & ~3;
-  if (S < 1 || S > kDecMaxSinks || cs * S > 4 * kDecThreads || c > 8 * kDecThreads) return false;
-  if (L - (cs - 1) * c < S) return false;          // the last share holds at least S columns
-  *chunk = c;
-  *kpt = 8;
-  return true;
+// Whether the cluster's fused top-S (decode_sink_topk) serves S sinks over L columns with
+// cs CTAs: S group maxima per CTA at most 4 x 128, and the cs * S candidates in CTA 0.
+bool plan_sink_topk(int L, int S, int cs) {
+  return S >= 1 && S <= kDecMaxSinks && S <= L && cs * S <= kSinkCand0;
 }
 
 template <int NQ, int STAGES, bool SPARSE, bool FUSED, bool COLSUM = false>
@@ -1262,7 +1364,7 @@ int run_decode(const DecArgs& a0, cudaStream_t stream, bool* sinks_done = nullpt
   }
   const int cs = choose_cluster<NQ, STAGES, SPARSE, FUSED, COLSUM>(units);
   if (COLSUM && a.sinks_out) {
-    if (!plan_sink_topk(a.L, a.S_out, cs, &a.ts_chunk, &a.ts_kpt)) a.sinks_out = nullptr;
+    if (!plan_sink_topk(a.L, a.S_out, cs)) a.sinks_out = nullptr;
     if (sinks_done) *sinks_done = a.sinks_out != nullptr;
   }
   auto kern = decode_attn_kernel<NQ, STAGES, SPARSE, FUSED, COLSUM>;

@@ -1,6 +1,6 @@
 """One-layer workload for kernel profiling (ncu) of a single Focus-dLLM call.
 
-  python -m diffusion_long_context_b200.profile_case --call sparse|fused|dense|colsum|select|blocks|means|refresh \
+  python -m diffusion_long_context_b200.profile_case --call sparse|fused|dense|colsum|select|blocks|means|refresh|entry \
       [--L 32768] [--repeat 3]
 
 Builds one layer of the 32K LLaDA-shaped step (synthetic, seeded), runs the whole step
@@ -21,7 +21,7 @@ from . import focus as F
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--call", default="sparse",
-                    choices=["sparse", "fused", "dense", "colsum", "select", "blocks", "means", "refresh"])
+                    choices=["sparse", "fused", "dense", "colsum", "select", "blocks", "means", "refresh", "entry"])
     ap.add_argument("--L", type=int, default=32768)
     ap.add_argument("--repeat", type=int, default=3)
     a = ap.parse_args()
@@ -75,16 +75,19 @@ def main():
     def refresh():
         F.focus_dense_attention(Qf, None, K, V, O_full, scale=1 / math.sqrt(c.d))
 
+    def entry():
+        F.focus_full_refresh(Qf, K, V, O_full, c.P, c.bs, kbar, scale=1 / math.sqrt(c.d))
+
     select()
     dense_colsum()
     means()
     blocks_sel()
     sparse()
     torch.cuda.synchronize()
-    if a.call == "refresh":
+    if a.call in ("refresh", "entry"):
         O_full = torch.empty((c.B, c.Hq, c.L, c.d), dtype=torch.bfloat16, device=dev)
     fn = {"sparse": sparse, "fused": fused, "dense": dense, "colsum": dense_colsum, "select": select, "blocks": blocks_sel,
-          "means": means, "refresh": refresh}[a.call]
+          "means": means, "refresh": refresh, "entry": entry}[a.call]
     for _ in range(a.repeat):
         fn()
     torch.cuda.synchronize()

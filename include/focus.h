@@ -183,10 +183,9 @@ FOCUS_API int focus_full_refresh(const focus_bf16* Q, const focus_bf16* K, const
  * ascending, -1 tail (as focus_sink_identify). Where the few-query kernel serves the shape
  * (d = 128, (Hq/Hkv) * qcap <= 64) the attention and the column sums run in one launch:
  * after the cluster merge the kernel re-reads the K tiles, most recently read first, for
- * the column sums. The same launch also selects the sinks within the cluster when each of
- * its CTAs holds at most 2560 columns (L up to about 10K with 4 CTAs per KV head, 20K with
- * 8) and S <= 512; otherwise the top-S runs as a second launch. Other shapes run the calls
- * in sequence. colsum and sinks are both written in every case. Requires 1 <= S <= 4096
+ * the column sums. The same launch also selects the sinks within the cluster when
+ * S <= 512, S <= L and (CTAs per KV head) x S <= 2048; otherwise the top-S runs as a
+ * second launch. Other shapes run the calls in sequence. colsum and sinks are both written in every case. Requires 1 <= S <= 4096
  * and the conditions of focus_dense_attention with column sums; ws/ws_bytes as there.
  */
 FOCUS_API int focus_dense_attention_sinks(const focus_bf16* Q, const int32_t* n_q, const focus_bf16* K,

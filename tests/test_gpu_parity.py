@@ -264,7 +264,8 @@ SINK_LAYER_CASES = [
     (2, 4, 4, 2500, 128, 32, [32, 7], 16),    # clusters of 8 CTAs
     (1, 8, 4, 1200, 128, 32, [27], 8),        # 64 rows per KV head: the 64-column kernel
     (1, 2, 1, 129, 128, 16, [16], 4),         # one partial key tile
-    (1, 4, 4, 300, 128, 32, [31], 120),       # the last share holds fewer than S columns: top-S kernel
+    (1, 4, 4, 300, 128, 32, [31], 120),       # S close to L: a CTA holds fewer than S columns
+    (1, 4, 4, 3000, 128, 32, [30], 300),      # S > 128: three group maxima per key lane
     (1, 2, 2, 5000, 128, 32, [32], 700),      # S beyond the cluster's candidate room: top-S kernel
     (1, 4, 4, 700, 64, 32, [25], 8),          # d = 64: tile kernel, column-sum kernel, top-S kernel
     (1, 28, 4, 900, 128, 32, [29], 16),       # 224 rows per KV head: tile kernel + column-sum kernel
@@ -292,6 +293,30 @@ def test_sink_layer_one_call(F, B, Hq, Hkv, L, d, qcap, n_q, S):
     np.testing.assert_allclose(colsum.cpu().double().numpy(), refC, rtol=2e-3, atol=1e-6)
     ties = assert_index_sets(sinks, refC, min(S, L), "sink layer sinks")
     assert ties == 0, f"{ties} near-tie sink sets"
+
+
+@pytest.mark.parametrize("L,S", [(12288, 32), (3000, 200)])
+def test_sink_layer_equal_column_sums(F, L, S):
+    """Degenerate case: K = 0 makes every score 0, so every column sum is n_q / L exactly
+    and the top-S is decided by the tie rule alone (the lowest columns). At 12288 columns
+    more columns tie than a CTA's candidate list holds, so each CTA takes the general radix
+    selection; at 3000 every column of a CTA is a candidate."""
+    B, Hq, Hkv, d, qcap = 1, 4, 4, 128, 32
+    Q = inputs.random_bf16((B, Hq, qcap, d), seed=77, device=DEV)
+    K = torch.zeros((B, Hkv, L, d), dtype=torch.bfloat16, device=DEV)
+    V = inputs.random_bf16((B, Hkv, L, d), seed=78, device=DEV)
+    nq = torch.tensor([29], dtype=torch.int32, device=DEV)
+    O = torch.empty((B, Hq, qcap, d), dtype=torch.bfloat16, device=DEV)
+    colsum = torch.empty((B, Hkv, L), dtype=torch.float32, device=DEV)
+    sinks = torch.full((B, Hkv, S), -7, dtype=torch.int32, device=DEV)
+    F.focus_dense_attention_sinks(Q, nq, K, V, O, colsum, sinks)
+    torch.cuda.synchronize()
+    assert F.device_error() == 0
+    c = colsum.cpu()
+    assert torch.all(c == c[0, 0, 0]), "column sums of equal scores differ"
+    np.testing.assert_allclose(float(c[0, 0, 0]) * L, 29.0, rtol=1e-4)
+    expect = torch.arange(S, dtype=torch.int32).expand(B, Hkv, S)
+    assert torch.equal(sinks.cpu(), expect)
 
 
 def test_sink_layer_cluster_top_s_matches_the_top_s_kernel(F):
