@@ -19,11 +19,6 @@
 // S_i only after PV_i(j) has read P_i). Each row keeps a reference maximum m: p = 2^(s - m)
 // while every s stays below m + 8; a tile that would exceed it moves m up and rescales the
 // row of O_i in tensor memory (after PV_i(j-1) has landed). Row sums are per-thread.
-// The two warpgroups take turns on the exponential unit (16 ex2 per clock per SM: a tile's
-// 2 x 16384 exponentials take about as many clocks as its four MMAs): warpgroup 1 starts the
-// exponentials of tile j once warpgroup 0 has finished its own, and warpgroup 0 those of
-// tile j + 1 once warpgroup 1 has finished tile j, so one warpgroup's exponentials overlap
-// the other's MMAs instead of both groups contending at once and then waiting together.
 //
 // Block entry (method steps (4): a prompt block is represented by the mean of its keys,
 // computed once per generation block): with kbar requested, the K tiles that stream through
@@ -65,7 +60,6 @@ struct __align__(8) RfBook {
   uint64_t k_full[kRfKStages], k_empty[kRfKStages];
   uint64_t v_full[kRfVStages], v_empty[kRfVStages];
   uint64_t s_full[2], p_full[2], o_done[2], drain;
-  uint64_t tok[2];         // exponential phase of a tile done by warpgroup 0 / 1
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -136,8 +130,6 @@ __global__ void __launch_bounds__(kRfThreads, 1)
         mbar_init(&bk->o_done[i], 1);
       }
       mbar_init(&bk->drain, 1);
-      mbar_init(&bk->tok[0], 4);
-      mbar_init(&bk->tok[1], 4);
       bk->abort_flag = 0;
       fence_mbar_init();
       tma_prefetch_desc(&tmQ);
@@ -352,15 +344,6 @@ __global__ void __launch_bounds__(kRfThreads, 1)
       }
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
       const float c2 = a.scale_log2;
-      // take turns on the exponential unit with the other warpgroup
-      if (wg == 1 || j > 0) {
-        const uint32_t par = static_cast<uint32_t>(wg == 1 ? j : j - 1) & 1u;
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&bk->tok[wg ^ 1], par, abort_flag, a.dev_err, DEV_ERR_TIMEOUT_SOFTMAX))) {
-          ok = false;
-          break;
-        }
-      }
       // P over the first 64 columns of S_i, 32 keys at a time. This thread has read its whole
       // row of S, and PV_i(j - 1), which read the previous P, completed before QK_i(j)
       // signalled s_full.
@@ -378,8 +361,6 @@ __global__ void __launch_bounds__(kRfThreads, 1)
         tmem_st16(tS + c * 16, pk);
       }
       const float ls = (lsc[0] + lsc[1]) + (lsc[2] + lsc[3]);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bk->tok[wg]);     // this tile's exponentials are done
       l_sum = l_sum * alpha + ls;
       if (j > 0 && __any_sync(0xffffffffu, rescale && alpha != 1.f)) {
         // O_i must hold PV_i(j - 1) before its rows are rescaled
