@@ -70,6 +70,7 @@ class SparseStep:
         sws = F.sparse_workspace_bytes(c.B, c.Hq, c.Hkv, c.L, c.d, c.acap, c.S, c.C, c.bs, c.P, c.g0, c.g1)
         self.ws = torch.empty(max(dws, sws, 256), dtype=torch.uint8, device=self.dev)
         self.graph: Optional[torch.cuda.CUDAGraph] = None
+        self.graph_io: Optional[torch.cuda.CUDAGraph] = None
         self.launches_per_step: Optional[int] = None
 
     # ------------------------------------------------------------------ inputs
@@ -187,8 +188,34 @@ class SparseStep:
         self.graph = g
         return g
 
+    def capture_io(self, conf_h: torch.Tensor, mask_h: torch.Tensor, outs):
+        """The step with its host traffic in one graph: the pinned host state (conf_h, mask_h)
+        is copied in, the step runs, and each (pinned host tensor, device tensor) pair of
+        `outs` is copied out, so that one replay_io() is one launch from the host."""
+        for t in (conf_h, mask_h, *(h for h, _ in outs)):
+            if not t.is_pinned():
+                raise ValueError("capture_io needs pinned host tensors")
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                self.conf_prev.copy_(conf_h, non_blocking=True)
+                self.mask.copy_(mask_h, non_blocking=True)
+                self.run()
+                for h, d in outs:
+                    h.copy_(d, non_blocking=True)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph_io = g
+        return g
+
     def replay(self):
         self.graph.replay()
 
+    def replay_io(self):
+        self.graph_io.replay()
+
     def release(self):
         self.graph = None
+        self.graph_io = None

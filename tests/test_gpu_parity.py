@@ -715,3 +715,37 @@ def test_sparse_step_sequencer(F, variant):
             assert np.array_equal(step.blocks[l].cpu().numpy(), ref["blocks"][l]), f"layer {l} blocks differ"
         assert_attention_close(step.O_active[l], ref["O"][l], rows_valid=nA, what=f"{variant} layer {l}")
     assert F.device_error() == 0
+
+
+def test_step_graph_with_host_io(F):
+    """SparseStep.capture_io: one graph holding the host-state copies in, the step and the
+    copies out gives the same host results as the step graph plus separate copies."""
+    from diffusion_long_context_b200 import configs as cf
+    from diffusion_long_context_b200.step import SparseStep
+    cfg = cf.scaled(cf.LLADA_8K, 1024, n_layers=4, Hq=4, Hkv=2, l_dense=1, C=4, S=8)
+    st = inputs.step_state(cfg)
+    layers = [inputs.make_layer(cfg, l, DEV, st.sink_pos) for l in range(cfg.n_layers)]
+    Q_full = torch.stack([lay[0] for lay in layers])
+    step = SparseStep(cfg, Q_full, [lay[1] for lay in layers], [lay[2] for lay in layers], device=DEV)
+    conf_h = torch.from_numpy(st.conf_prev).pin_memory()
+    mask_h = torch.from_numpy(st.mask).pin_memory()
+    step.set_state(conf_h, mask_h, non_blocking=False)
+    step.block_entry()
+    step.capture()
+    step.replay()
+    torch.cuda.synchronize()
+    ref_o, ref_a, ref_n = step.O_active[-1].cpu(), step.i_active.cpu(), step.n_active.cpu()
+    step.O_active[-1].zero_()
+    step.i_active.fill_(-5)
+    out_h = torch.full(ref_o.shape, 7.0, dtype=torch.bfloat16).pin_memory()
+    act_h = torch.full(ref_a.shape, -9, dtype=torch.int32).pin_memory()
+    nact_h = torch.zeros(ref_n.shape, dtype=torch.int32).pin_memory()
+    step.capture_io(conf_h, mask_h, [(out_h, step.O_active[-1]), (act_h, step.i_active), (nact_h, step.n_active)])
+    for _ in range(2):
+        step.replay_io()
+        torch.cuda.current_stream().synchronize()
+    assert torch.equal(act_h, ref_a) and torch.equal(nact_h, ref_n)
+    # the cluster's tiles are claimed dynamically, so the last bits of O may differ
+    torch.testing.assert_close(out_h.float(), ref_o.float(), rtol=0, atol=1e-2)
+    step.release()
+    assert F.device_error() == 0
