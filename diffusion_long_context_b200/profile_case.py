@@ -1,6 +1,6 @@
 """One-layer workload for kernel profiling (ncu) of a single Focus-dLLM call.
 
-  python -m diffusion_long_context_b200.profile_case --call sparse|fused|dense|colsum|select|blocks|means|refresh|entry \
+  python -m diffusion_long_context_b200.profile_case --call sparse|fused|dense|colsum|sinks|select|blocks|means|refresh|entry \
       [--L 32768] [--repeat 3]
 
 Builds one layer of the 32K LLaDA-shaped step (synthetic, seeded), runs the whole step
@@ -21,7 +21,8 @@ from . import focus as F
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--call", default="sparse",
-                    choices=["sparse", "fused", "dense", "colsum", "select", "blocks", "means", "refresh", "entry"])
+                    choices=["sparse", "fused", "dense", "colsum", "sinks", "select", "blocks", "means", "refresh",
+                             "entry"])
     ap.add_argument("--L", type=int, default=32768)
     ap.add_argument("--repeat", type=int, default=3)
     a = ap.parse_args()
@@ -57,6 +58,9 @@ def main():
         F.focus_dense_attention(Qa, n_active, K, V, O, colsum=colsum, ws=ws)
         F.focus_sink_identify(colsum, c.S, sinks)
 
+    def sink_layer():
+        F.focus_dense_attention_sinks(Qa, n_active, K, V, O, colsum, sinks, ws=ws)
+
     def means():
         F.focus_block_means(K, c.P, c.bs, kbar)
 
@@ -87,7 +91,7 @@ def main():
     if a.call in ("refresh", "entry"):
         O_full = torch.empty((c.B, c.Hq, c.L, c.d), dtype=torch.bfloat16, device=dev)
     fn = {"sparse": sparse, "fused": fused, "dense": dense, "colsum": dense_colsum, "select": select, "blocks": blocks_sel,
-          "means": means, "refresh": refresh, "entry": entry}[a.call]
+          "means": means, "refresh": refresh, "entry": entry, "sinks": sink_layer}[a.call]
     for _ in range(a.repeat):
         fn()
     torch.cuda.synchronize()
