@@ -584,6 +584,8 @@ FUSED_CASES = [
     ("gqa7_sliced", 1, 28, 4, 1024, 32, 1100, 64, 6, 8, 32, [31]),       # 224 rows: four row slices
     ("gqa3_b2", 2, 6, 2, 1024, 32, 1100, 64, 7, 5, 32, [32, 12]),         # 96 rows: two slices
     ("gqa16_two_calls", 1, 16, 1, 1024, 32, 1100, 64, 6, 8, 32, [31]),   # 512 rows: two-call path
+    # the fused kernel's limits: 4096 blocks (nb), C = 512, S = 512, 64 rows (NQ = 64)
+    ("max_nb_c_s", 1, 2, 1, 32768, 32, 32800, 8, 512, 512, 32, [32]),
 ]
 
 
