@@ -293,12 +293,6 @@ __device__ __forceinline__ float2 dsmem_ld_v2(uint32_t addr) {
   asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
   return v;
 }
-__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-
 // Named barrier with an OR reduction of `pred` over the `nthreads` participants.
 __device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred) {
   uint32_t r;
