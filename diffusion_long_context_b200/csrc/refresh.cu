@@ -94,6 +94,27 @@ __device__ __forceinline__ bool rf_wait_drain(uint64_t* bar, uint32_t parity) {
   return true;
 }
 
+// fp32 pairs (f32x2): one instruction forms the exponent arguments of two keys, and one
+// adds two probabilities to two of the row-sum chains
+__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 __global__ void __launch_bounds__(kRfThreads, 1)
     refresh_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ RfArgs a) {
@@ -347,20 +368,26 @@ __global__ void __launch_bounds__(kRfThreads, 1)
       // P over the first 64 columns of S_i, 32 keys at a time. This thread has read its whole
       // row of S, and PV_i(j - 1), which read the previous P, completed before QK_i(j)
       // signalled s_full.
-      float lsc[4] = {0.f, 0.f, 0.f, 0.f};           // four independent row-sum chains
+      const unsigned long long c2x2 = f2_pack(c2, c2), nm2 = f2_pack(neg_m, neg_m);
+      unsigned long long lsc2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};   // four row-sum chains
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float p0 = exp2_approx(fmaf(sv[32 * c + 2 * k], c2, neg_m));
-          const float p1 = exp2_approx(fmaf(sv[32 * c + 2 * k + 1], c2, neg_m));
-          lsc[k & 3] += p0 + p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sv[32 * c + 2 * k], sv[32 * c + 2 * k + 1]), c2x2, nm2), x0, x1);
+          const float p0 = exp2_approx(x0);
+          const float p1 = exp2_approx(x1);
+          lsc2[k & 1] = f2_add(lsc2[k & 1], f2_pack(p0, p1));
           pk[k] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + c * 16, pk);
       }
-      const float ls = (lsc[0] + lsc[1]) + (lsc[2] + lsc[3]);
+      float l0, l1, l2, l3;
+      f2_unpack(lsc2[0], l0, l1);
+      f2_unpack(lsc2[1], l2, l3);
+      const float ls = (l0 + l2) + (l1 + l3);
       l_sum = l_sum * alpha + ls;
       if (j > 0 && __any_sync(0xffffffffu, rescale && alpha != 1.f)) {
         // O_i must hold PV_i(j - 1) before its rows are rescaled
